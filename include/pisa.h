@@ -1,0 +1,146 @@
+/*
+ * pisa.h — C ABI of a B200 (sm_100a) library for piecewise sparse attention (PISA).
+ *
+ * Method: "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion Transformers"
+ * (gist.science technical summary of arXiv 2602.01077), §2 방법론.  Key/value tokens of each
+ * (batch, head) are cut into contiguous blocks of `block` tokens (the last may be shorter).  For
+ * each query block i the router splits the key blocks into critical blocks S_i, attended exactly,
+ * and the rest U_i, which still enter the same softmax numerator N_t and denominator D_t through
+ *     alpha_{t,j} = exp(s q_t . kbar_j)                  (zeroth order, per block)
+ *     N_t += sum_{j in U_i} alpha_{t,j} vsum_j + s (q_t Hbar) sum_{j in U_i} alpha_{t,j}
+ *     D_t += sum_{j in U_i} cnt_j alpha_{t,j}
+ * and o_t = N_t / D_t.  s is `softmax_scale`.
+ *
+ * Conventions shared by every entry point
+ *   - q, k, v and o are dense row-major [B, H, L, d] tensors (d = head_dim for keys and values).
+ *     They share one element type (`dtype`); o has the type of q.
+ *   - Every pointer argument is a DEVICE pointer on the current CUDA device unless it is a
+ *     `const pisa_shape*` / `pisa_stats*` (host structs) or documented otherwise.  The caller owns
+ *     all memory; the library never allocates or frees device memory and keeps no pointer after a
+ *     call returns.
+ *   - Device pointers must be 16-byte aligned.  All work is enqueued on `stream` (0 = legacy
+ *     default stream) and is asynchronous; the call returns once the kernels are enqueued.
+ *   - Arguments are validated before anything is enqueued.  A call that returns an error status
+ *     has enqueued nothing and written nothing.
+ *   - No exceptions cross the ABI.  The library keeps no mutable host state apart from a cache of
+ *     device attributes and resolved driver entry points.
+ *   - Supported on the GPU: dtype PISA_BF16 with head_dim 128 and block 64 or 128 (tensor-core
+ *     path), and PISA_FP32 with head_dim 64 or 128 and block 64 or 128 (fp32 FMA path).
+ */
+#ifndef PISA_H_
+#define PISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* pisa_stream_t;
+
+typedef enum {
+  PISA_OK = 0,
+  PISA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad size, keep_k or lambda out of range */
+  PISA_ERR_UNSUPPORTED = 2,    /* valid shape the GPU kernels do not implement (e.g. head_dim 96) */
+  PISA_ERR_CUDA = 3,           /* a CUDA launch or driver call failed */
+  PISA_ERR_DEVICE_TIMEOUT = 4  /* a kernel's bounded wait ran out (reported by pisa_read_device_error) */
+} pisa_status;
+
+typedef enum { PISA_BF16 = 0, PISA_FP32 = 1 } pisa_dtype;
+
+/* PISA_MODE_EXACT_ONLY drops U_i entirely (the keep-or-drop sparse attention the method is
+ * compared against, §1 문제 정의); it needs keep_k >= 1. */
+typedef enum { PISA_MODE_PISA = 0, PISA_MODE_EXACT_ONLY = 1 } pisa_mode;
+
+typedef struct {
+  int32_t batch;          /* B >= 1 */
+  int32_t heads;          /* H >= 1 */
+  int32_t seq_len;        /* L >= 1 */
+  int32_t head_dim;       /* d */
+  int32_t block;          /* tokens per key block and per query block */
+  int32_t dtype;          /* pisa_dtype of q, k, v, o */
+  float   softmax_scale;  /* s: multiplies every logit and the first-order correction */
+} pisa_shape;
+
+/* Per-head block statistics written by pisa_precompute.  nb = pisa_num_blocks(L, block).
+ * All fp32 arrays are dense row-major.  The *_op arrays are tensor-core operand copies and are
+ * used (and must be non-null) only when dtype == PISA_BF16. */
+typedef struct {
+  float* qbar;     /* [B,H,nb,d]  mean of q over query block i                                */
+  float* kbar;     /* [B,H,nb,d]  centroid of key block j                                      */
+  float* vsum;     /* [B,H,nb,d]  sum of values of block j                                     */
+  float* hbar;     /* [B,H,d,d]   Hbar[a][c]: mean over j of H_j, H_j = sum_n (k_n-kbar_j)^T v_n */
+  float* M;        /* [B,H,nb]    ||H_j - Hbar||_F                                             */
+  float* H;        /* nullable [B,H,nb,d,d]: per-block H_j, written only when non-null         */
+  void*  kbar_op;  /* bf16 [B,H,nb,d]  kbar rounded to bf16                                    */
+  void*  vsum_op;  /* bf16 [B,H,nb,d]  vsum rounded to bf16                                    */
+  void*  hbar_op;  /* bf16 [B,H,d,d]   softmax_scale * Hbar^T, i.e. hbar_op[c][a]              */
+} pisa_stats;
+
+/* ABI revision of this header. */
+int32_t pisa_abi_version(void);
+
+/* nb = ceil(seq_len / block), or -1 if either argument is < 1. */
+int32_t pisa_num_blocks(int32_t seq_len, int32_t block);
+
+/* Bytes of one contiguous buffer that pisa_stats_carve can split into every pisa_stats array
+ * (H included when with_H != 0).  0 if the shape is invalid. */
+size_t pisa_stats_bytes(const pisa_shape* shape, int32_t with_H);
+
+/* Host-only pointer arithmetic: fills *out with 256-byte-aligned sub-ranges of [base, base+bytes).
+ * base must be 256-byte aligned; bytes >= pisa_stats_bytes(shape, with_H).  Enqueues nothing. */
+pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, int32_t with_H,
+                             pisa_stats* out);
+
+/* Device scratch bytes needed by pisa_precompute and pisa_attention for this shape (the first 256
+ * bytes hold the device status word read by pisa_read_device_error). */
+size_t pisa_workspace_bytes(const pisa_shape* shape);
+
+/* Pre-computation (§2 하드웨어 구현, step 1; zeroth-order and global first-order bullets of
+ * 핵심 알고리즘; M_j from 공분산 인식 라우팅): from q, k, v writes every array of *stats.
+ * ws: device scratch of at least pisa_workspace_bytes(shape), contents need not be initialised.
+ * Deterministic: fixed-order reductions, no floating-point atomics. */
+pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                            const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream);
+
+/* Covariance-aware top-k routing (§2 공분산 인식 라우팅):
+ *   s_ij = softmax_scale * qbar_i . kbar_j
+ *   P_ij = cnt_j exp(s_ij) / sum_l cnt_l exp(s_il)
+ *   r_ij = P_ij + lambda * M_j / sum_l M_l        (the M term is 0 when every M_j is 0)
+ * sel    [B,H,nb,keep_k] int32: the keep_k largest r_ij of row i, ties to the lower j, ascending.
+ * order  nullable [B,H,nb] int32: a permutation of the query blocks of each head that puts blocks
+ *        with similar selections next to each other (pisa_attention runs consecutive pairs of it as
+ *        one 128-row tile when block == 64; it changes no result).
+ * scores nullable [B,H,nb,nb] fp32: r_ij.
+ * Requires 0 <= keep_k <= nb, lambda finite and >= 0, nb <= 4096. */
+pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,
+                       int32_t* sel, int32_t* order, float* scores, pisa_stream_t stream);
+
+/* Exact-or-approximate attention (§2: o_t = N_t / D_t and the numerator equation; 하드웨어 구현
+ * stages 1-3: exact selected blocks, zeroth-order scan of the other blocks, global first-order
+ * correction).  sel as written by pisa_route (ascending, distinct, < nb; checked on the device,
+ * a bad entry sets the status word).  order: nullable, as written by pisa_route; null means
+ * 0, 1, ..., nb-1.  o: [B,H,L,d] of dtype.  mode: pisa_mode.  ws as for pisa_precompute. */
+pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                           const pisa_stats* stats, const int32_t* sel, const int32_t* order,
+                           int32_t keep_k, int32_t mode, void* o, void* ws, size_t ws_bytes,
+                           pisa_stream_t stream);
+
+/* Synchronises `stream`, copies the device status word out of ws into *code (0 = clean; otherwise
+ * a PISA_DEVERR_* value below) and clears it.  Returns PISA_ERR_DEVICE_TIMEOUT when a bounded wait
+ * ran out, PISA_ERR_INVALID_ARG for a bad selection entry, PISA_OK when clean. */
+pisa_status pisa_read_device_error(void* ws, int32_t* code, pisa_stream_t stream);
+
+#define PISA_DEVERR_WAIT_TIMEOUT 1   /* an mbarrier wait exceeded its iteration limit */
+#define PISA_DEVERR_BAD_SELECTION 2  /* sel held an entry out of range or out of order */
+
+/* Static description of a status code. */
+const char* pisa_status_string(pisa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PISA_H_ */

@@ -1,0 +1,79 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that some pin catches each one.
+
+A mistake that no pin notices would mean the pins do not constrain that part of the oracle.
+"""
+import numpy as np
+import pytest
+
+from oracle import pisa_oracle as O
+from tests import oracle_pins as P
+
+
+def _corr_sign(qi, stats, alpha, U, scale, first_order):
+    return -_ORIG["_correction"](qi, stats, alpha, U, scale, first_order)
+
+
+def _corr_zero(qi, stats, alpha, U, scale, first_order):
+    return 0.0 * _ORIG["_correction"](qi, stats, alpha, U, scale, first_order)
+
+
+def _corr_transposed(qi, stats, alpha, U, scale, first_order):
+    st = dict(stats)
+    st["Hbar"] = stats["Hbar"].T
+    st["H"] = np.swapaxes(stats["H"], 1, 2)
+    return _ORIG["_correction"](qi, st, alpha, U, scale, first_order)
+
+
+def _corr_unscaled(qi, stats, alpha, U, scale, first_order):
+    return _ORIG["_correction"](qi, stats, alpha, U, 1.0, first_order)
+
+
+MUTATIONS = {
+    "correction dropped": ("_correction", _corr_zero),
+    "correction sign flipped": ("_correction", _corr_sign),
+    "correction uses H transposed": ("_correction", _corr_transposed),
+    "correction misses softmax scale": ("_correction", _corr_unscaled),
+    "denominator misses cnt_j": ("_denominator", lambda ez, a, c: ez.sum(axis=1) + a.sum(axis=1)),
+    "H_j not centred": ("_first_order_matrix", lambda kk, vv, kbar: kk.T @ vv),
+    "Hbar is a sum": ("_global_first_order", lambda H: H.sum(axis=0)),
+    "centroid is first token": ("_centroid", lambda kk: kk[0].copy()),
+    "value sum is a mean": ("_value_sum", lambda vv: vv.mean(axis=0)),
+    "route mass ignores cnt": ("_block_attention_mass",
+                               lambda qb, kb, cnt, s: _ORIG["_block_attention_mass"](qb, kb, np.ones_like(cnt), s)),
+    "M not normalised": ("_normalised_cov", lambda M: M),
+    "M squared": ("_cov_norm", lambda Hj, Hb, norm: _ORIG["_cov_norm"](Hj, Hb, norm) ** 2),
+}
+_ORIG = {name: getattr(O, name) for name, _ in MUTATIONS.values()}
+
+
+def _tie_high(r, keep_k):
+    nqb, nb = r.shape
+    out = np.zeros((nqb, keep_k), dtype=np.int64)
+    for i in range(nqb):
+        order = np.lexsort((-np.arange(nb), -r[i]))
+        out[i] = np.sort(order[:keep_k])
+    return out
+
+
+MUTATIONS["ties to the higher index"] = ("route_select", _tie_high)
+_ORIG["route_select"] = O.route_select
+
+
+def _caught():
+    failed = []
+    for pin in P.ALL_PINS:
+        try:
+            ok, _ = pin()
+        except Exception:          # a crash under the planted mistake counts as a catch
+            ok = False
+        if not ok:
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = _caught()
+    assert failed, f"no pin caught the planted mistake: {name}"

@@ -1,0 +1,350 @@
+"""Benchmark of the PISA hot path (pre-compute -> route -> attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one pass of the three calls over one batch of synthetic, device-resident input.  The
+metric is effective TFLOP/s (FLOPs of the exactly-attended, selected blocks only) per step, summed
+over ranks; each rank runs its own batch element (weak scaling, no data-path collective).  Rank 0
+prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample
+of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective TFLOP/s and ms per attention call (B200, 87.5% sparsity) vs dense"
+DEFAULT_WORKLOAD = "video-dit-large"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def effective_flops(sel, order_blocks_L: int, block: int, d: int, nb: int):
+    """(exact FLOPs of selected blocks, centroid FLOPs of unselected blocks) for sel [B,H,nqb,k]."""
+    import torch
+    B, H, nqb, k = sel.shape
+    L = order_blocks_L
+    cnt = torch.full((nb,), block, dtype=torch.float64, device=sel.device)
+    cnt[-1] = L - (nb - 1) * block
+    sel_cnt = cnt[sel.long()].sum(-1) if k > 0 else torch.zeros((B, H, nqb), dtype=torch.float64, device=sel.device)
+    n_i = cnt  # query block sizes use the same partition
+    exact = float((4.0 * d * n_i[None, None, :] * sel_cnt).sum())
+    centroid = float(4.0 * d * (n_i.sum() * (nb - k)) * B * H)
+    return exact, centroid
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from piecewise_approximate_attention_b200 import _lib as C
+    from piecewise_approximate_attention_b200.runtime import Pisa
+    from piecewise_approximate_attention_b200.workloads import WORKLOADS, make_qkv
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    # each rank runs its own batch element: seed offset by rank
+    q, k, v = make_qkv(w, seed=w.seed + rank)
+    B, H, L, d = q.shape
+    p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        qd, kd, vd = (x.to(dev, non_blocking=False) for x in (q, k, v))
+        o = torch.empty_like(qd)
+    torch.cuda.synchronize()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        p.precompute(qd, kd, vd, stream)
+        if evs:
+            evs[1].record(stream)
+        p.route(stream=stream)
+        if evs:
+            evs[2].record(stream)
+        p.attention(qd, kd, vd, o, stream=stream)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, code = p.device_error(stream)
+    if st != C.PISA_OK:
+        raise RuntimeError(f"device status {st} code {code} after warm-up")
+
+    per = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t0.record(stream)
+    for s in range(args.steps):
+        step(per[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t0.elapsed_time(t1)
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in per)
+    route_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in per)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in per)
+    st, code = p.device_error(stream)
+    if st != C.PISA_OK:
+        raise RuntimeError(f"device status {st} code {code} after timing")
+
+    exact_fl, centroid_fl = effective_flops(p.sel, L, w.block, d, p.nb)
+    corr_fl = 2.0 * L * d * d * B * H
+    ms_step = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step, attn_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_step, attn_ms_max = t.tolist()
+    else:
+        attn_ms_max = attn_ms
+
+    # library's own dense path (keep_k = nb) and exact-only mode, same GPU, outside the timed region
+    dense = Pisa(B, H, L, d, w.block, p.nb, w.lam, w.dtype, 1.0, dev, pair=False)
+    dense.precompute(qd, kd, vd, stream)
+    dense.route(stream=stream)
+
+    def time_calls(fn, n=3):
+        fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    o2 = torch.empty_like(o)
+    dense_ms = time_calls(lambda: dense.attention(qd, kd, vd, o2, stream=stream))
+    exact_only_ms = time_calls(lambda: p.attention(qd, kd, vd, o2, mode=C.PISA_MODE_EXACT_ONLY, stream=stream))
+    dense_fl = 4.0 * L * L * d * B * H
+    del dense
+
+    # end to end through the public API with host buffers: H2D of q, k, v and D2H of o every step
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(q).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+        step()
+        with torch.cuda.stream(stream):
+            oh.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = t.item()
+
+    peak, peak_sus, hbm, peak_kind = _peaks()
+    attn_alg = exact_fl + centroid_fl + corr_fl
+    achieved = attn_alg / (attn_ms * 1e-3) / 1e12
+    result = {
+        "metric": METRIC,
+        "value": round(world * exact_fl / (ms_step * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (smooth 3D field + N(0,1) noise, seeded; stands in for Wan2.1-class video DiT activations)",
+        "config": {"workload": w.name, "batch_per_gpu": B, "heads": H, "seq_len": L, "head_dim": d,
+                   "block": w.block, "keep_k": w.keep_k, "num_blocks": p.nb, "sparsity": w.sparsity,
+                   "lambda": w.lam, "parallelism": f"weak, 1 batch element per GPU x {world}",
+                   "l2": "inputs (3 x %.0f MB) larger than L2; no flush" % (q.numel() * q.element_size() / 1e6)},
+        "ms_per_attention_call": round(attn_ms_max, 4),
+        "ms_precompute": round(pre_ms, 4),
+        "ms_route": round(route_ms, 4),
+        "dense_ms_per_attention_call": round(dense_ms, 4),
+        "dense_tflops": round(dense_fl / (dense_ms * 1e-3) / 1e12, 3),
+        "speedup_vs_dense_attention": round(dense_ms / attn_ms, 3),
+        "exact_only_ms_per_attention_call": round(exact_only_ms, 4),
+        "attention_overhead_vs_exact_only": round(attn_ms / exact_only_ms - 1.0, 4),
+        "effective_tflops_attention_only": round(exact_fl / (attn_ms * 1e-3) / 1e12, 3),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "pisa_attention", "peak_kind": f"{peak_kind} bf16 dense burst",
+                     "frac_of_sustained": round(achieved / peak_sus, 4),
+                     "algorithmic_flops_per_launch": attn_alg},
+        "e2e": {"value": round(world * exact_fl / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                "d2h_bytes_per_step": o.numel() * o.element_size()},
+        "gpu_launches": args.steps * p.launches_per_step(),
+        "clocks": clk,
+    }
+    if rank == 0:
+        result["cpu_baseline"] = cpu_baseline(w)
+    return result
+
+
+def cpu_baseline(w, heads=(0,)):
+    """fp64 oracle on a bounded sample (one full head of the workload) on the host cores."""
+    import numpy as np
+    import threadpoolctl
+    from oracle import pisa_oracle as O
+    from piecewise_approximate_attention_b200.workloads import make_qkv
+    cores = len(os.sched_getaffinity(0))
+    q, k, v = (t.double().numpy() for t in make_qkv(w, heads=list(heads)))
+    with threadpoolctl.threadpool_limits(cores):
+        t = time.perf_counter()
+        res = O.pisa(q, k, v, w.block, w.keep_k, w.lam)
+        dt = time.perf_counter() - t
+    sel = res["sel"]
+    L, d, b = w.seq_len, w.head_dim, w.block
+    nb = w.num_blocks
+    cnt = np.full(nb, b, dtype=np.float64)
+    cnt[-1] = L - (nb - 1) * b
+    exact = float((4.0 * d * cnt[None, None, :] * cnt[sel].sum(-1)).sum()) if w.keep_k else 0.0
+    return {"value": round(exact / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"{len(heads)} of {w.heads} heads of {w.name} (full pre-compute, routing and attention), fp64 numpy"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from piecewise_approximate_attention_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    vals = []
+    for _ in range(args.warmup):
+        pass   # the oracle has no warm-up state; warm-up steps are not repeated on the CPU
+    cb = None
+    for _ in range(max(1, args.steps)):
+        cb = cpu_baseline(w)
+        vals.append(cb["value"])
+    v = statistics.median(vals)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": {"workload": w.name},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import datetime
+    import torch
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -33,6 +33,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define PISA_API __attribute__((visibility("default")))
+#else
+#define PISA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -80,29 +86,31 @@ typedef struct {
 } pisa_stats;
 
 /* ABI revision of this header. */
-int32_t pisa_abi_version(void);
+PISA_API int32_t pisa_abi_version(void);
 
 /* nb = ceil(seq_len / block), or -1 if either argument is < 1. */
-int32_t pisa_num_blocks(int32_t seq_len, int32_t block);
+PISA_API int32_t pisa_num_blocks(int32_t seq_len, int32_t block);
 
 /* Bytes of one contiguous buffer that pisa_stats_carve can split into every pisa_stats array
  * (H included when with_H != 0).  0 if the shape is invalid. */
-size_t pisa_stats_bytes(const pisa_shape* shape, int32_t with_H);
+PISA_API size_t pisa_stats_bytes(const pisa_shape* shape, int32_t with_H);
 
 /* Host-only pointer arithmetic: fills *out with 256-byte-aligned sub-ranges of [base, base+bytes).
  * base must be 256-byte aligned; bytes >= pisa_stats_bytes(shape, with_H).  Enqueues nothing. */
-pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, int32_t with_H,
+PISA_API pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, int32_t with_H,
                              pisa_stats* out);
 
 /* Device scratch bytes needed by pisa_precompute and pisa_attention for this shape (the first 256
  * bytes hold the device status word read by pisa_read_device_error). */
-size_t pisa_workspace_bytes(const pisa_shape* shape);
+PISA_API size_t pisa_workspace_bytes(const pisa_shape* shape);
 
 /* Pre-computation (§2 하드웨어 구현, step 1; zeroth-order and global first-order bullets of
  * 핵심 알고리즘; M_j from 공분산 인식 라우팅): from q, k, v writes every array of *stats.
- * ws: device scratch of at least pisa_workspace_bytes(shape), contents need not be initialised.
- * Deterministic: fixed-order reductions, no floating-point atomics. */
-pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
+ * ws: device scratch of at least pisa_workspace_bytes(shape).  Its first 256 bytes hold the device
+ * status word, which must be zero before the first call (allocate ws zeroed) and is cleared by
+ * pisa_read_device_error; the rest need not be initialised.  Calls that share one ws must not run
+ * concurrently.  Deterministic: fixed-order reductions, no floating-point atomics. */
+PISA_API pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
                             const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream);
 
 /* Covariance-aware top-k routing (§2 공분산 인식 라우팅):
@@ -115,7 +123,7 @@ pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* 
  *        one 128-row tile when block == 64; it changes no result).
  * scores nullable [B,H,nb,nb] fp32: r_ij.
  * Requires 0 <= keep_k <= nb, lambda finite and >= 0, nb <= 4096. */
-pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,
+PISA_API pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,
                        int32_t* sel, int32_t* order, float* scores, pisa_stream_t stream);
 
 /* Exact-or-approximate attention (§2: o_t = N_t / D_t and the numerator equation; 하드웨어 구현
@@ -123,7 +131,7 @@ pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t
  * correction).  sel as written by pisa_route (ascending, distinct, < nb; checked on the device,
  * a bad entry sets the status word).  order: nullable, as written by pisa_route; null means
  * 0, 1, ..., nb-1.  o: [B,H,L,d] of dtype.  mode: pisa_mode.  ws as for pisa_precompute. */
-pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k, const void* v,
+PISA_API pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k, const void* v,
                            const pisa_stats* stats, const int32_t* sel, const int32_t* order,
                            int32_t keep_k, int32_t mode, void* o, void* ws, size_t ws_bytes,
                            pisa_stream_t stream);
@@ -131,13 +139,13 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
 /* Synchronises `stream`, copies the device status word out of ws into *code (0 = clean; otherwise
  * a PISA_DEVERR_* value below) and clears it.  Returns PISA_ERR_DEVICE_TIMEOUT when a bounded wait
  * ran out, PISA_ERR_INVALID_ARG for a bad selection entry, PISA_OK when clean. */
-pisa_status pisa_read_device_error(void* ws, int32_t* code, pisa_stream_t stream);
+PISA_API pisa_status pisa_read_device_error(void* ws, int32_t* code, pisa_stream_t stream);
 
 #define PISA_DEVERR_WAIT_TIMEOUT 1   /* an mbarrier wait exceeded its iteration limit */
 #define PISA_DEVERR_BAD_SELECTION 2  /* sel held an entry out of range or out of order */
 
 /* Static description of a status code. */
-const char* pisa_status_string(pisa_status status);
+PISA_API const char* pisa_status_string(pisa_status status);
 
 #ifdef __cplusplus
 }

@@ -177,16 +177,21 @@ def _denominator(ez: np.ndarray, alpha: np.ndarray, cnt_u: np.ndarray) -> np.nda
 
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, sel: np.ndarray,
                    stats: Dict, scale: float = 1.0, mode: str = "pisa",
-                   first_order: str = "global") -> np.ndarray:
-    """o = N / D for one head; ``mode='exact_only'`` drops U_i (the keep-or-drop baseline)."""
+                   first_order: str = "global", qblocks: Optional[Sequence[int]] = None) -> np.ndarray:
+    """o = N / D for one head; ``mode='exact_only'`` drops U_i (the keep-or-drop baseline).
+
+    ``qblocks`` restricts the evaluation to those query blocks (other rows are NaN).
+    """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     L = q.shape[0]
     bounds = block_bounds(L, block)
     nb = len(bounds)
-    o = np.zeros((L, v.shape[1]))
-    for i, (qs, qe) in enumerate(bounds):
+    o = np.zeros((L, v.shape[1])) if qblocks is None else np.full((L, v.shape[1]), np.nan)
+    wanted = range(nb) if qblocks is None else sorted(set(int(i) for i in qblocks))
+    for i in wanted:
+        qs, qe = bounds[i]
         S = [int(j) for j in sel[i]]
         Sset = set(S)
         U = [j for j in range(nb) if j not in Sset] if mode == "pisa" else []
@@ -211,11 +216,14 @@ def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, sel:
 
 
 def pisa(q, k, v, block: int, keep_k: int, lam: float, scale: float = 1.0, mode: str = "pisa",
-         first_order: str = "global", norm: str = "fro", heads: Optional[Sequence[int]] = None) -> Dict:
+         first_order: str = "global", norm: str = "fro", heads: Optional[Sequence[int]] = None,
+         qblocks: Optional[Sequence[int]] = None) -> Dict:
     """Whole pipeline on [B, H, L, d] inputs: stats -> route -> attention, per (batch, head).
 
     Returns dict with o [B,H,L,dv], sel [B,H,nqb,keep_k], scores r [B,H,nqb,nb] and the stats
-    arrays stacked over (B, H).  ``heads`` restricts the work to a subset of head indices.
+    arrays stacked over (B, H).  ``heads`` selects which head indices of the input to evaluate;
+    ``qblocks`` restricts the attention output to those query blocks (statistics and routing are
+    always complete).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -229,7 +237,7 @@ def pisa(q, k, v, block: int, keep_k: int, lam: float, scale: float = 1.0, mode:
             st = block_stats(q[b, h], k[b, h], v[b, h], block, norm)
             r = route_scores(st, lam, scale)
             sel = route_select(r, keep_k)
-            o = attention_head(q[b, h], k[b, h], v[b, h], block, sel, st, scale, mode, first_order)
+            o = attention_head(q[b, h], k[b, h], v[b, h], block, sel, st, scale, mode, first_order, qblocks)
             for key, val in (("o", o), ("sel", sel), ("r", r), ("qbar", st["qbar"]), ("kbar", st["kbar"]),
                              ("vsum", st["vsum"]), ("Hbar", st["Hbar"]), ("M", st["M"]), ("cnt", st["cnt"])):
                 row[key].append(val)

@@ -1,0 +1,196 @@
+// Host entry points of the C ABI declared in pisa.h: validation, buffer carving, dispatch.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace pisa {
+namespace {
+
+constexpr int kMaxBlocks = 4096;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the shape; fills g.  Returns INVALID_ARG for impossible shapes and UNSUPPORTED for
+// shapes the GPU kernels do not implement.
+pisa_status check_shape(const pisa_shape* s, Dims* g) {
+  if (!s) return PISA_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->heads < 1 || s->seq_len < 1 || s->head_dim < 1 || s->block < 1)
+    return PISA_ERR_INVALID_ARG;
+  if (s->dtype != PISA_BF16 && s->dtype != PISA_FP32) return PISA_ERR_INVALID_ARG;
+  if (!std::isfinite(s->softmax_scale)) return PISA_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
+  if (s->block != 64 && s->block != 128) return PISA_ERR_UNSUPPORTED;
+  const long long nb = ((long long)s->seq_len + s->block - 1) / s->block;
+  if (nb > kMaxBlocks) return PISA_ERR_UNSUPPORTED;
+  if ((long long)s->batch * s->heads > 65535) return PISA_ERR_UNSUPPORTED;
+  g->B = s->batch;
+  g->H = s->heads;
+  g->L = s->seq_len;
+  g->d = s->head_dim;
+  g->block = s->block;
+  g->nb = (int)nb;
+  g->dtype = s->dtype;
+  g->scale = s->softmax_scale;
+  return PISA_OK;
+}
+
+pisa_status check_stats(const Dims& g, const pisa_stats* st, bool need_ops) {
+  if (!st) return PISA_ERR_INVALID_ARG;
+  const void* req[] = {st->qbar, st->kbar, st->vsum, st->hbar, st->M};
+  for (const void* p : req)
+    if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
+  if (st->H && !aligned16(st->H)) return PISA_ERR_INVALID_ARG;
+  if (need_ops && g.dtype == PISA_BF16) {
+    const void* ops[] = {st->kbar_op, st->vsum_op, st->hbar_op};
+    for (const void* p : ops)
+      if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
+  }
+  return PISA_OK;
+}
+
+pisa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PISA_OK : PISA_ERR_CUDA; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Sizes of the stats arrays in carve order.
+void stats_sizes(const Dims& g, int with_H, size_t out[9]) {
+  const size_t bh = (size_t)g.BH(), nb = (size_t)g.nb, d = (size_t)g.d;
+  out[0] = bh * nb * d * 4;            // qbar
+  out[1] = bh * nb * d * 4;            // kbar
+  out[2] = bh * nb * d * 4;            // vsum
+  out[3] = bh * d * d * 4;             // hbar
+  out[4] = bh * nb * 4;                // M
+  out[5] = with_H ? bh * nb * d * d * 4 : 0;  // H
+  out[6] = bh * nb * d * 2;            // kbar_op
+  out[7] = bh * nb * d * 2;            // vsum_op
+  out[8] = bh * d * d * 2;             // hbar_op
+}
+
+}  // namespace
+}  // namespace pisa
+
+using namespace pisa;
+
+extern "C" {
+
+int32_t pisa_abi_version(void) { return 1; }
+
+int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
+  if (seq_len < 1 || block < 1) return -1;
+  return (int32_t)(((long long)seq_len + block - 1) / block);
+}
+
+size_t pisa_stats_bytes(const pisa_shape* shape, int32_t with_H) {
+  Dims g;
+  if (check_shape(shape, &g) != PISA_OK) return 0;
+  size_t sz[9];
+  stats_sizes(g, with_H, sz);
+  size_t tot = 0;
+  for (size_t s : sz) tot += round_up(s, 256);
+  return tot;
+}
+
+pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, int32_t with_H, pisa_stats* out) {
+  Dims g;
+  pisa_status s = check_shape(shape, &g);
+  if (s != PISA_OK) return s;
+  if (!base || !out || (reinterpret_cast<uintptr_t>(base) & 255u)) return PISA_ERR_INVALID_ARG;
+  if (bytes < pisa_stats_bytes(shape, with_H)) return PISA_ERR_INVALID_ARG;
+  size_t sz[9];
+  stats_sizes(g, with_H, sz);
+  char* p = static_cast<char*>(base);
+  void* ptr[9];
+  for (int i = 0; i < 9; ++i) {
+    ptr[i] = sz[i] ? p : nullptr;
+    p += round_up(sz[i], 256);
+  }
+  pisa_stats st;
+  st.qbar = static_cast<float*>(ptr[0]);
+  st.kbar = static_cast<float*>(ptr[1]);
+  st.vsum = static_cast<float*>(ptr[2]);
+  st.hbar = static_cast<float*>(ptr[3]);
+  st.M = static_cast<float*>(ptr[4]);
+  st.H = static_cast<float*>(ptr[5]);
+  st.kbar_op = ptr[6];
+  st.vsum_op = ptr[7];
+  st.hbar_op = ptr[8];
+  *out = st;
+  return PISA_OK;
+}
+
+size_t pisa_workspace_bytes(const pisa_shape* shape) {
+  Dims g;
+  if (check_shape(shape, &g) != PISA_OK) return 0;
+  return kStatusBytes + round_up(partials_bytes(g), 256);
+}
+
+pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                            const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+  Dims g;
+  pisa_status s = check_shape(shape, &g);
+  if (s != PISA_OK) return s;
+  if (!q || !k || !v || !ws || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(ws))
+    return PISA_ERR_INVALID_ARG;
+  if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
+  if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
+  return cuda_status(launch_precompute_simt(g, q, k, v, *stats, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,
+                       int32_t* sel, int32_t* order, float* scores, pisa_stream_t stream) {
+  Dims g;
+  pisa_status s = check_shape(shape, &g);
+  if (s != PISA_OK) return s;
+  if ((s = check_stats(g, stats, false)) != PISA_OK) return s;
+  if (keep_k < 0 || keep_k > g.nb || !std::isfinite(lambda) || lambda < 0.f) return PISA_ERR_INVALID_ARG;
+  if ((keep_k > 0 && (!sel || !aligned16(sel))) || (order && !aligned16(order)) || (scores && !aligned16(scores)))
+    return PISA_ERR_INVALID_ARG;
+  return cuda_status(launch_route(g, *stats, keep_k, lambda, sel, order, scores,
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                           const pisa_stats* stats, const int32_t* sel, const int32_t* order, int32_t keep_k,
+                           int32_t mode, void* o, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+  Dims g;
+  pisa_status s = check_shape(shape, &g);
+  if (s != PISA_OK) return s;
+  if (!q || !k || !v || !o || !ws || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(ws))
+    return PISA_ERR_INVALID_ARG;
+  if (mode != PISA_MODE_PISA && mode != PISA_MODE_EXACT_ONLY) return PISA_ERR_INVALID_ARG;
+  if (keep_k < 0 || keep_k > g.nb || (mode == PISA_MODE_EXACT_ONLY && keep_k < 1)) return PISA_ERR_INVALID_ARG;
+  if (keep_k > 0 && (!sel || !aligned16(sel))) return PISA_ERR_INVALID_ARG;
+  if (order && !aligned16(order)) return PISA_ERR_INVALID_ARG;
+  if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
+  if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
+  int* status = static_cast<int*>(ws);
+  return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+pisa_status pisa_read_device_error(void* ws, int32_t* code, pisa_stream_t stream) {
+  if (!ws || !code || !aligned16(ws)) return PISA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t host = 0;
+  if (cudaMemcpyAsync(&host, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess) return PISA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return PISA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PISA_ERR_CUDA;
+  *code = host;
+  if (host == 0) return PISA_OK;
+  return host == PISA_DEVERR_WAIT_TIMEOUT ? PISA_ERR_DEVICE_TIMEOUT : PISA_ERR_INVALID_ARG;
+}
+
+const char* pisa_status_string(pisa_status status) {
+  switch (status) {
+    case PISA_OK: return "ok";
+    case PISA_ERR_INVALID_ARG: return "invalid argument";
+    case PISA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PISA_ERR_CUDA: return "CUDA error";
+    case PISA_ERR_DEVICE_TIMEOUT: return "device-side bounded wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// Shared device/host definitions of the PISA library (internal; not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "pisa.h"
+
+namespace pisa {
+
+// Problem dimensions after validation.
+struct Dims {
+  int B, H, L, d, block, nb, dtype;
+  float scale;
+  int BH() const { return B * H; }
+  int last_cnt() const { return L - (nb - 1) * block; }
+};
+
+// Workspace layout: [0, 256) device status word(s); [256, ...) precompute partial sums of H_j.
+constexpr size_t kStatusBytes = 256;
+constexpr int kBlocksPerPart = 16;   // key blocks whose H_j one precompute CTA sums
+
+inline int num_parts(const Dims& g) { return (g.nb + kBlocksPerPart - 1) / kBlocksPerPart; }
+inline size_t partials_bytes(const Dims& g) {
+  return (size_t)g.BH() * num_parts(g) * g.d * g.d * sizeof(float);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Records the first device-side error code; later codes do not overwrite it.
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ int block_count(int j, int L, int block) {
+  int s = j * block;
+  int e = s + block < L ? s + block : L;
+  return e - s;
+}
+
+// ---- launchers (defined in the kernel translation units) ----
+cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,
+                                   const pisa_stats& st, void* ws, cudaStream_t stream);
+cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
+                         int32_t* order, float* scores, cudaStream_t stream);
+cudaError_t launch_attention_simt(const Dims& g, const void* q, const void* k, const void* v,
+                                  const pisa_stats& st, const int32_t* sel, int keep_k, int mode,
+                                  void* o, int* status, cudaStream_t stream);
+
+}  // namespace pisa

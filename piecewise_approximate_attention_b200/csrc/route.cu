@@ -1,0 +1,285 @@
+// Covariance-aware top-k routing and the query-block pairing order.
+//
+// "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion Transformers", §2 방법론,
+// 공분산 인식 라우팅: the block selection score combines the attention score with the block
+// covariance norm M_j = ||H_j - Hbar||; blocks of high relevance or high heterogeneity are computed
+// exactly, smoother ones are left to the Taylor terms.  Per query block i (fp32 throughout, so that
+// near-ties resolve like the fp64 definition up to ~1e-6 relative):
+//   s_ij = scale * qbar_i . kbar_j
+//   P_ij = cnt_j exp(s_ij - max_l s_il) / sum_l cnt_l exp(s_il - max_l s_il)
+//   r_ij = P_ij + lambda * M_j / sum_l M_l
+//   S_i  = keep_k largest r_ij, ties to the lower j, written in ascending j.
+// Top-k is an exact radix select on the IEEE bit patterns of r (r >= 0, so bit order is value
+// order) followed by an ordered warp compaction; no sort is needed.
+#include "common.cuh"
+
+namespace pisa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRows = 4;          // query blocks per CTA
+
+__device__ __forceinline__ float warp_max(float x) {
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Selects the keep_k largest keys of u[0..nb) (ties to the lower index) and writes their indices,
+// ascending, to out.  Runs on one warp; hist is a private 256-entry scratch.
+__device__ void warp_topk(const uint32_t* u, int nb, int keep_k, uint32_t* hist, int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  if (keep_k <= 0) return;
+  uint32_t prefix = 0, pmask = 0;
+  int want = keep_k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < nb; j += 32)
+      if ((u[j] & pmask) == prefix) atomicAdd(&hist[(u[j] >> shift) & 255u], 1u);
+    __syncwarp();
+    // lane l owns digits 255-8l .. 248-8l (descending); find the digit where the count of keys
+    // with a larger-or-equal digit first reaches `want`.
+    uint32_t cnt[8];
+    uint32_t tot = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) { cnt[t] = hist[255 - 8 * lane - t]; tot += cnt[t]; }
+    uint32_t incl = tot;
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - tot;
+    int found_digit = -1;
+    uint32_t above = 0;
+    if (excl < (uint32_t)want && incl >= (uint32_t)want) {
+      uint32_t run = excl;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (found_digit < 0 && run + cnt[t] >= (uint32_t)want) { found_digit = 255 - 8 * lane - t; above = run; }
+        run += cnt[t];
+      }
+    }
+    const unsigned owner = __ballot_sync(0xffffffffu, found_digit >= 0);
+    const int src = __ffs(owner) - 1;
+    found_digit = __shfl_sync(0xffffffffu, found_digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    want -= (int)above;
+    prefix |= (uint32_t)found_digit << shift;
+    pmask |= 255u << shift;
+    __syncwarp();
+  }
+  // prefix is now the exact key of the keep_k-th largest element; `want` of its equals are taken.
+  const unsigned lt = (1u << lane) - 1u;
+  int pos = 0, eq_seen = 0;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < nb ? u[j] : 0u;
+    const bool gt = j < nb && key > prefix;
+    const bool eq = j < nb && key == prefix;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eqm & lt) < want);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[pos + __popc(tm & lt)] = j;
+    pos += __popc(tm);
+    eq_seen += __popc(eqm);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
+                                                         const float* __restrict__ M, int L, int block, int nb,
+                                                         float scale, int keep_k, float lam,
+                                                         int32_t* __restrict__ sel, float* __restrict__ scores) {
+  extern __shared__ float smem[];
+  float* qs = smem;                                        // [kRows][D]
+  float* r = qs + kRows * D;                               // [kRows][nb]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(r + kRows * nb);   // [kWarps][256]
+  float* red = reinterpret_cast<float*>(hist + kWarps * 256);     // [kWarps]
+  const int bh = blockIdx.y, i0 = blockIdx.x * kRows;
+  const int rows = min(kRows, nb - i0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* Mh = M + (size_t)bh * nb;
+
+  for (int idx = threadIdx.x; idx < kRows * D; idx += kThreads) {
+    const int ri = idx / D;
+    qs[idx] = ri < rows ? scale * qbar[((size_t)bh * nb + i0 + ri) * D + idx % D] : 0.f;
+  }
+  // sum_l M_l in a fixed order
+  float msum = 0.f;
+  for (int j = threadIdx.x; j < nb; j += kThreads) msum += Mh[j];
+  msum = warp_sum(msum);
+  if (lane == 0) red[warp] = msum;
+  __syncthreads();
+  msum = 0.f;
+  for (int w = 0; w < kWarps; ++w) msum += red[w];
+  const float minv = msum > 0.f ? lam / msum : 0.f;
+
+  const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nb * D);
+  for (int j = threadIdx.x; j < nb; j += kThreads) {
+    float acc[kRows];
+#pragma unroll
+    for (int ri = 0; ri < kRows; ++ri) acc[ri] = 0.f;
+    for (int a4 = 0; a4 < D / 4; ++a4) {
+      const float4 kv = kb4[(size_t)j * (D / 4) + a4];
+#pragma unroll
+      for (int ri = 0; ri < kRows; ++ri) {
+        const float* qq = qs + ri * D + 4 * a4;
+        acc[ri] = fmaf(qq[0], kv.x, fmaf(qq[1], kv.y, fmaf(qq[2], kv.z, fmaf(qq[3], kv.w, acc[ri]))));
+      }
+    }
+#pragma unroll
+    for (int ri = 0; ri < kRows; ++ri) r[ri * nb + j] = acc[ri];
+  }
+  __syncthreads();
+
+  const float last_cnt = (float)(L - (nb - 1) * block);
+  for (int ri = warp; ri < rows; ri += kWarps) {
+    float* rr = r + ri * nb;
+    float mx = -INFINITY;
+    for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, rr[j]);
+    mx = warp_max(mx);
+    float den = 0.f;
+    for (int j = lane; j < nb; j += 32) {
+      const float w = (j == nb - 1 ? last_cnt : (float)block) * expf(rr[j] - mx);
+      rr[j] = w;
+      den += w;
+    }
+    den = warp_sum(den);
+    const float inv = 1.f / den;
+    const size_t row = (size_t)bh * nb + i0 + ri;
+    for (int j = lane; j < nb; j += 32) {
+      const float val = rr[j] * inv + minv * Mh[j];
+      rr[j] = val;
+      if (scores) scores[row * nb + j] = val;
+    }
+    __syncwarp();
+    warp_topk(reinterpret_cast<const uint32_t*>(rr), nb, keep_k, hist + warp * 256, sel + row * keep_k);
+  }
+}
+
+// Query-block pairing for 128-row tiles when block == 64: a greedy pass in index order pairs
+// each unpaired query block i with the unpaired block p in (i, i + kWin] whose selection shares
+// the most key blocks with S_i (ties to the nearer p).  Blocks left without a partner go last.
+// The attention result does not depend on the order; only the union of S_i and S_p, which one
+// tile iterates over, does.  One CTA per head; bitmaps of the selections live in shared memory.
+constexpr int kWin = 128;
+constexpr int kChunk = 64;
+
+__global__ void __launch_bounds__(kThreads) pair_kernel(const int32_t* __restrict__ sel, int nb, int keep_k,
+                                                        int32_t* __restrict__ order) {
+  extern __shared__ uint32_t psm[];
+  const int nwords = (nb + 31) / 32;
+  uint32_t* bits = psm;                                            // [kChunk + kWin][nwords]
+  uint16_t* ov = reinterpret_cast<uint16_t*>(bits + (kChunk + kWin) * nwords);  // [kChunk][kWin]
+  uint32_t* used = reinterpret_cast<uint32_t*>(ov + kChunk * kWin);             // [nwords]
+  int32_t* singles = reinterpret_cast<int32_t*>(used + nwords);                 // [nb]
+  __shared__ int npos, nsingle;
+  const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t* S = sel + (size_t)bh * nb * keep_k;
+  int32_t* out = order + (size_t)bh * nb;
+  for (int w = threadIdx.x; w < nwords; w += kThreads) used[w] = 0u;
+  if (threadIdx.x == 0) { npos = 0; nsingle = 0; }
+  for (int c0 = 0; c0 < nb; c0 += kChunk) {
+    const int nrows = min(nb - c0, kChunk + kWin);
+    __syncthreads();
+    for (int e = threadIdx.x; e < (kChunk + kWin) * nwords; e += kThreads) bits[e] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < nrows * keep_k; e += kThreads) {
+      const int r = e / keep_k;
+      const int j = S[(size_t)(c0 + r) * keep_k + e % keep_k];
+      if (j >= 0 && j < nb) atomicOr(&bits[r * nwords + (j >> 5)], 1u << (j & 31));
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kChunk * kWin; e += kThreads) {
+      const int a = e / kWin, dl = e % kWin + 1;
+      int cnt = 0;
+      if (a + dl < nrows) {
+        const uint32_t* x = bits + a * nwords;
+        const uint32_t* y = bits + (a + dl) * nwords;
+        for (int w = 0; w < nwords; ++w) cnt += __popc(x[w] & y[w]);
+      }
+      ov[e] = (uint16_t)cnt;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      for (int a = 0; a < kChunk && c0 + a < nb; ++a) {
+        const int i = c0 + a;
+        if ((used[i >> 5] >> (i & 31)) & 1u) continue;
+        int best = -1, bestv = -1;
+        for (int dl = lane + 1; dl <= kWin; dl += 32) {
+          const int p = i + dl;
+          if (p < nb && !((used[p >> 5] >> (p & 31)) & 1u)) {
+            const int val = ov[a * kWin + dl - 1];
+            if (val > bestv) { bestv = val; best = dl; }
+          }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          const int ov2 = __shfl_xor_sync(0xffffffffu, bestv, o);
+          const int ob2 = __shfl_xor_sync(0xffffffffu, best, o);
+          if (ov2 > bestv || (ov2 == bestv && ob2 >= 0 && (best < 0 || ob2 < best))) { bestv = ov2; best = ob2; }
+        }
+        if (lane == 0) {
+          used[i >> 5] |= 1u << (i & 31);
+          if (best > 0) {
+            const int p = i + best;
+            used[p >> 5] |= 1u << (p & 31);
+            out[npos] = i;
+            out[npos + 1] = p;
+            npos += 2;
+          } else {
+            singles[nsingle++] = i;
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < nsingle; e += kThreads) out[npos + e] = singles[e];
+}
+
+__global__ void identity_order(int nb, int32_t* __restrict__ order) {
+  const int bh = blockIdx.y;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nb; i += gridDim.x * blockDim.x)
+    order[(size_t)bh * nb + i] = i;
+}
+
+}  // namespace
+
+cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
+                         int32_t* order, float* scores, cudaStream_t stream) {
+  const size_t smem = ((size_t)kRows * g.d + (size_t)kRows * g.nb) * sizeof(float) + kWarps * 256 * sizeof(uint32_t) +
+                      kWarps * sizeof(float);
+  dim3 grid((g.nb + kRows - 1) / kRows, g.BH());
+  cudaError_t e;
+  if (g.d == 64) {
+    if ((e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+    route_kernel<64><<<grid, kThreads, smem, stream>>>(st.qbar, st.kbar, st.M, g.L, g.block, g.nb, g.scale, keep_k,
+                                                        lam, sel, scores);
+  } else {
+    if ((e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+    route_kernel<128><<<grid, kThreads, smem, stream>>>(st.qbar, st.kbar, st.M, g.L, g.block, g.nb, g.scale, keep_k,
+                                                         lam, sel, scores);
+  }
+  if ((e = cudaGetLastError())) return e;
+  if (order) {
+    if (g.block == 64 && keep_k > 0 && g.nb > 2) {
+      const int nwords = (g.nb + 31) / 32;
+      const size_t psmem = (size_t)(kChunk + kWin) * nwords * 4 + (size_t)kChunk * kWin * 2 + (size_t)nwords * 4 +
+                           (size_t)g.nb * 4;
+      if ((e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem))) return e;
+      pair_kernel<<<g.BH(), kThreads, psmem, stream>>>(sel, g.nb, keep_k, order);
+    } else {
+      identity_order<<<dim3((g.nb + 255) / 256, g.BH()), 256, 0, stream>>>(g.nb, order);
+    }
+    if ((e = cudaGetLastError())) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace pisa

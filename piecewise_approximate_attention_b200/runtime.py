@@ -1,0 +1,60 @@
+"""Buffers and call sequence for one PISA attention shape (pre-compute -> route -> attention).
+
+All three steps run in the CUDA library through the C ABI; this module only allocates device
+memory with torch and passes pointers and the current stream.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+from . import _lib as C
+
+
+class Pisa:
+    """Reusable PISA attention for a fixed [B, H, L, d] shape, block size, keep_k and lambda.
+
+    ``pair=True`` asks the router for the query-block pairing order used by 128-row tiles when
+    block == 64 (a scheduling choice: the output does not depend on it).
+    """
+
+    def __init__(self, batch: int, heads: int, seq_len: int, head_dim: int, block: int, keep_k: int,
+                 lam: float, dtype: str = "bf16", softmax_scale: float = 1.0, device="cuda",
+                 mode: int = C.PISA_MODE_PISA, with_H: bool = False, pair: bool = True):
+        import torch
+        self.shape = C.make_shape(batch, heads, seq_len, head_dim, block, dtype, softmax_scale)
+        self.block, self.keep_k, self.lam, self.mode = block, keep_k, lam, mode
+        self.nb = C.pisa_num_blocks(seq_len, block)
+        self.device = torch.device(device)
+        self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.stats = C.alloc_stats(self.shape, self.device, with_H)
+        self.ws = C.alloc_workspace(self.shape, self.device)
+        self.sel = torch.empty((batch, heads, self.nb, max(keep_k, 1)), dtype=torch.int32, device=self.device)
+        self.order = torch.empty((batch, heads, self.nb), dtype=torch.int32, device=self.device) if pair else None
+
+    def precompute(self, q, k, v, stream=None):
+        C.pisa_precompute(self.shape, q, k, v, self.stats, self.ws, stream)
+
+    def route(self, scores=None, stream=None):
+        C.pisa_route(self.shape, self.stats, self.keep_k, self.lam, self.sel, self.order, scores, stream)
+
+    def attention(self, q, k, v, o, sel=None, order=None, mode: Optional[int] = None, stream=None):
+        s = self.sel if sel is None else sel
+        od = self.order if order is None else order
+        C.pisa_attention(self.shape, q, k, v, self.stats, s, od, self.keep_k, self.mode if mode is None else mode,
+                         o, self.ws, stream)
+
+    def __call__(self, q, k, v, o=None, stream=None):
+        import torch
+        if o is None:
+            o = torch.empty_like(q)
+        self.precompute(q, k, v, stream)
+        self.route(stream=stream)
+        self.attention(q, k, v, o, stream=stream)
+        return o
+
+    def launches_per_step(self) -> int:
+        """Kernels one __call__ enqueues: pre-compute 3, routing 1 (+1 pairing), attention 1."""
+        return 3 + 1 + (1 if self.order is not None else 0) + 1
+
+    def device_error(self, stream=None):
+        return C.pisa_read_device_error(self.ws, stream)

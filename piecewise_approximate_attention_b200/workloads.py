@@ -97,10 +97,10 @@ def _field(rng: np.random.Generator, grid: Tuple[int, int, int], d: int) -> np.n
              + omega[:, 1, None, None, None] * y[None, None, :, None]
              + omega[:, 2, None, None, None] * x[None, None, None, :])
     theta = (2.0 * math.pi) * theta.reshape(4, -1)                     # [4, Limg]
-    F = np.zeros((theta.shape[1], d), dtype=np.float64)
-    for m in range(4):
-        F += amp[m][None, :] * np.sin(theta[m][:, None] + phi[m][None, :])
-    return F * (2.0 ** -0.5)
+    # sin(theta + phi) = sin(theta) cos(phi) + cos(theta) sin(phi): one [Limg x 8] @ [8 x d] product
+    basis = np.concatenate([np.sin(theta), np.cos(theta)], axis=0).T   # [Limg, 8]
+    coef = np.concatenate([amp * np.cos(phi), amp * np.sin(phi)], axis=0)  # [8, d]
+    return (basis @ coef) * (2.0 ** -0.5)
 
 
 def make_head(w: Workload, b: int, h: int, seed: Optional[int] = None):

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared symbol, and rejects
+invalid arguments before touching the GPU.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from piecewise_approximate_attention_b200 import _lib as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pisa.h")).read()
+    return sorted(set(re.findall(r"PISA_API\s+[\w\s\*]*?\b(pisa_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.lib()
+    names = _declared()
+    assert len(names) >= 10
+    assert set(names) == set(C.SYMBOLS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_and_blocks():
+    assert C.lib().pisa_abi_version() == 1
+    assert C.pisa_num_blocks(32760, 64) == 512
+    assert C.pisa_num_blocks(75600, 128) == 591
+    assert C.pisa_num_blocks(1, 64) == 1
+    assert C.pisa_num_blocks(0, 64) == -1
+    assert C.pisa_num_blocks(10, 0) == -1
+
+
+def test_status_strings():
+    for s in range(5):
+        assert C.status_string(s)
+    assert "unknown" in C.status_string(99)
+
+
+def _shape(**kw):
+    base = dict(batch=1, heads=2, seq_len=1000, head_dim=128, block=64, dtype="bf16", softmax_scale=1.0)
+    base.update(kw)
+    return C.make_shape(**base)
+
+
+def test_stats_bytes_and_carve_are_host_only():
+    sh = _shape()
+    n0 = C.pisa_stats_bytes(sh, False)
+    n1 = C.pisa_stats_bytes(sh, True)
+    nb = 16
+    assert n1 - n0 >= 2 * nb * 128 * 128 * 4
+    st = C.PisaStats()
+    base = 1 << 20      # never dereferenced: carving is pointer arithmetic
+    assert C.lib().pisa_stats_carve(ctypes.byref(sh), base, n1, 1, ctypes.byref(st)) == C.PISA_OK
+    ptrs = [st.qbar, st.kbar, st.vsum, st.hbar, st.M, st.H, st.kbar_op, st.vsum_op, st.hbar_op]
+    assert all(p and p % 256 == 0 and base <= p < base + n1 for p in ptrs)
+    assert len(set(ptrs)) == len(ptrs)
+    assert C.lib().pisa_stats_carve(ctypes.byref(sh), base + 16, n1, 1, ctypes.byref(st)) == C.PISA_ERR_INVALID_ARG
+    assert C.lib().pisa_stats_carve(ctypes.byref(sh), base, n1 - 1, 1, ctypes.byref(st)) == C.PISA_ERR_INVALID_ARG
+    assert C.pisa_workspace_bytes(sh) >= 256 + 2 * 1 * 128 * 128 * 4
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(head_dim=96), C.PISA_ERR_UNSUPPORTED),
+    (dict(block=32), C.PISA_ERR_UNSUPPORTED),
+    (dict(seq_len=0), C.PISA_ERR_INVALID_ARG),
+    (dict(batch=0), C.PISA_ERR_INVALID_ARG),
+    (dict(dtype=7), C.PISA_ERR_INVALID_ARG),
+    (dict(softmax_scale=float("nan")), C.PISA_ERR_INVALID_ARG),
+    (dict(seq_len=64 * 4097), C.PISA_ERR_UNSUPPORTED),
+])
+def test_bad_shapes_rejected(kw, expect):
+    sh = _shape(**kw)
+    st = C.PisaStats()
+    assert C.lib().pisa_precompute(ctypes.byref(sh), 16, 16, 16, ctypes.byref(st), 16, 1 << 30, None) == expect
+    assert C.pisa_stats_bytes(sh, False) == 0
+    assert C.pisa_workspace_bytes(sh) == 0
+
+
+def _fake_stats(sh):
+    st = C.PisaStats()
+    n = C.pisa_stats_bytes(sh, False)
+    assert C.lib().pisa_stats_carve(ctypes.byref(sh), 1 << 24, n, 0, ctypes.byref(st)) == C.PISA_OK
+    return st
+
+
+def test_invalid_arguments_rejected_without_launch():
+    L = C.lib()
+    sh = _shape()
+    st = _fake_stats(sh)
+    ws = C.pisa_workspace_bytes(sh)
+    P = 1 << 28
+    bs = ctypes.byref(sh)
+    # null / misaligned tensors
+    assert L.pisa_precompute(bs, None, P, P, ctypes.byref(st), P, ws, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_precompute(bs, P + 4, P, P, ctypes.byref(st), P, ws, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_precompute(bs, P, P, P, ctypes.byref(st), P, ws - 1, None) == C.PISA_ERR_INVALID_ARG
+    bad = C.PisaStats.from_buffer_copy(st)
+    bad.kbar_op = None
+    assert L.pisa_precompute(bs, P, P, P, ctypes.byref(bad), P, ws, None) == C.PISA_ERR_INVALID_ARG
+    # routing arguments
+    assert L.pisa_route(bs, ctypes.byref(st), 17, 0.5, P, None, None, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_route(bs, ctypes.byref(st), -1, 0.5, P, None, None, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_route(bs, ctypes.byref(st), 4, -0.1, P, None, None, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_route(bs, ctypes.byref(st), 4, float("inf"), P, None, None, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_route(bs, ctypes.byref(st), 4, 0.5, None, None, None, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_route(bs, ctypes.byref(st), 4, 0.5, P + 8, None, None, None) == C.PISA_ERR_INVALID_ARG
+    # attention arguments
+    att = lambda keep, mode, sel=P, o=P, wsb=ws: L.pisa_attention(bs, P, P, P, ctypes.byref(st), sel, None, keep,
+                                                                  mode, o, P, wsb, None)
+    assert att(4, 2) == C.PISA_ERR_INVALID_ARG
+    assert att(0, C.PISA_MODE_EXACT_ONLY) == C.PISA_ERR_INVALID_ARG
+    assert att(17, C.PISA_MODE_PISA) == C.PISA_ERR_INVALID_ARG
+    assert att(4, C.PISA_MODE_PISA, sel=None) == C.PISA_ERR_INVALID_ARG
+    assert att(4, C.PISA_MODE_PISA, o=None) == C.PISA_ERR_INVALID_ARG
+    assert att(4, C.PISA_MODE_PISA, wsb=100) == C.PISA_ERR_INVALID_ARG
+    code = ctypes.c_int32()
+    assert L.pisa_read_device_error(None, ctypes.byref(code), None) == C.PISA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(C, "_lib", None)
+    monkeypatch.setattr(C, "_LIB_PATH", "/nonexistent/libpisa_b200.so")
+    with pytest.raises(RuntimeError, match="not built"):
+        C.lib()

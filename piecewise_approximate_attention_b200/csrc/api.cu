@@ -20,6 +20,7 @@ pisa_status check_shape(const pisa_shape* s, Dims* g) {
   if (s->dtype != PISA_BF16 && s->dtype != PISA_FP32) return PISA_ERR_INVALID_ARG;
   if (!std::isfinite(s->softmax_scale)) return PISA_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
+  if (s->dtype == PISA_BF16 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
   if (s->block != 64 && s->block != 128) return PISA_ERR_UNSUPPORTED;
   const long long nb = ((long long)s->seq_len + s->block - 1) / s->block;
   if (nb > kMaxBlocks) return PISA_ERR_UNSUPPORTED;
@@ -166,8 +167,19 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
   if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
   if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   int* status = static_cast<int*>(ws);
-  return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (g.dtype == PISA_BF16) {
+    AttnMaps maps;
+    const uint64_t bh = (uint64_t)g.BH();
+    if (!encode_bf16_3d(&maps.q, q, g.d, g.L, bh, g.block) || !encode_bf16_3d(&maps.k, k, g.d, g.L, bh, g.block) ||
+        !encode_bf16_3d(&maps.v, v, g.d, g.L, bh, g.block) ||
+        !encode_bf16_3d(&maps.kbar, stats->kbar_op, g.d, g.nb, bh, 128) ||
+        !encode_bf16_3d(&maps.vsum, stats->vsum_op, g.d, g.nb, bh, 128) ||
+        !encode_bf16_3d(&maps.hbar, stats->hbar_op, g.d, g.d, bh, 128))
+      return PISA_ERR_CUDA;
+    return cuda_status(launch_attention_sm100(g, maps, sel, order, keep_k, mode, o, status, kWaitLimitNs, cs));
+  }
+  return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status, cs));
 }
 
 pisa_status pisa_read_device_error(void* ws, int32_t* code, pisa_stream_t stream) {

@@ -1,0 +1,505 @@
+// Fused exact-or-approximate attention for sm_100a: TMA + tcgen05 (TMEM accumulators).
+//
+// "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion Transformers", §2 방법론,
+// 하드웨어 구현: one FlashAttention-style online softmax interleaves
+//   stage 1  exact attention over the selected key blocks S_i (loaded to on-chip memory),
+//   stage 2  the zeroth-order scan of the unselected blocks: logits q_t . kbar_j against the block
+//            centroids and values sum_n v_n, with denominator weight cnt_j,
+//   stage 3  the global first-order correction s (q_t Hbar) sum_{j in U_i} alpha_tj, injected before
+//            the division o_t = N_t / D_t.
+//
+// Mapping onto B200 (one CTA = one 128-row query tile; two CTAs share an SM):
+//   * Q tile 128 x 128 bf16 in shared memory (two 64-column 128B-swizzled halves, filled by TMA).
+//     With 64-token blocks a tile holds two query blocks a, b (consecutive entries of the router's
+//     pairing order); with 128-token blocks it holds one.
+//   * The tile walks a list of 128-row "key tiles": first the union of S_a and S_b (two 64-token key
+//     blocks per tile, each half masked for the query block that did not select it), then, in PISA
+//     mode, ceil(nb/128) centroid tiles (kbar_j as keys, vsum_j as values; columns of selected blocks
+//     masked).  Both kinds run through the same tcgen05 MMAs: S = Q K^T into TMEM (fp32), softmax in
+//     registers (one thread per row), P (bf16) written back over S in TMEM, O += P V with P read from
+//     TMEM and V from shared memory (MN-major).
+//   * The running max is updated lazily (only when it grows by more than 2^8), so O in TMEM is
+//     rescaled rarely; all terms of N_t and D_t carry the same max, so the result is unchanged.
+//   * The correction is one more MMA, Q (s Hbar^T), into the S columns after the last PV; the
+//     epilogue computes o = (O + A * (Q s Hbar)) / l with A = sum of alpha over U_i.
+// Warp roles: warps 0-3 softmax + epilogue (TMEM lanes 0-127), warp 4 TMA producer, warp 5 MMA
+// issuer and TMEM owner.  Every mbarrier wait is bounded; a timeout sets the status word and the
+// CTA drains its own in-flight work, frees TMEM and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace pisa {
+namespace {
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int kThreads = 192;
+constexpr int kHalf = 128 * 64 * 2;        // one 128-row x 64-column bf16 half: 16 KB
+constexpr int kTileBytes = 2 * kHalf;      // 32 KB
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColO = 128;
+constexpr int kWords = 128;                // selection bitmap words (nb <= 4096)
+
+struct alignas(1024) Smem {
+  uint8_t v[kTileBytes];
+  uint8_t q[kTileBytes];
+  uint8_t k[kTileBytes];
+  uint64_t bar_q, bar_kfull, bar_kempty, bar_vfull, bar_vempty, bar_sfull, bar_pfull, bar_odone, bar_final, bar_drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_exact, n_cent, need_corr;
+  uint32_t bitsA[kWords];
+  uint32_t bitsB[kWords];
+};
+
+struct Params {
+  int L, nb, block, keep_k, mode, dense;
+  float scale_log2;
+  const int32_t* sel;
+  const int32_t* order;
+  __nv_bfloat16* o;
+  int* status;
+  unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ bool bit_of(const uint32_t* bits, int j) { return (bits[j >> 5] >> (j & 31)) & 1u; }
+
+// Ascending enumeration of the key blocks in S_a | S_b.  The producer and every softmax thread run
+// identical copies, so the key-tile sequence needs no hand-off between roles.
+struct UnionIter {
+  int w = 0;
+  uint32_t cur = 0;
+  __device__ __forceinline__ int next(const uint32_t* a, const uint32_t* b) {
+    while (cur == 0) {
+      if (w >= kWords) return -1;
+      cur = a[w] | b[w];
+      ++w;
+    }
+    const int j = (w - 1) * 32 + __ffs(cur) - 1;
+    cur &= cur - 1;
+    return j;
+  }
+};
+
+// Key tile t: kind 0 = exact (key blocks j0, j1; j1 = -1 when absent or block == 128),
+// kind 1 = centroid tile starting at centroid j0.
+struct KeyTile {
+  int kind, j0, j1;
+};
+__device__ __forceinline__ KeyTile key_tile(int t, int n_exact, bool pair, UnionIter& it, const uint32_t* a,
+                                            const uint32_t* b) {
+  KeyTile kt;
+  if (t < n_exact) {
+    kt.kind = 0;
+    kt.j0 = it.next(a, b);
+    kt.j1 = pair ? it.next(a, b) : -1;
+  } else {
+    kt.kind = 1;
+    kt.j0 = (t - n_exact) * 128;
+    kt.j1 = -1;
+  }
+  return kt;
+}
+
+__device__ __forceinline__ bool wait_or_abort(Smem& sm, uint64_t* bar, uint32_t parity, const Params& p) {
+  if (mbar_wait_bounded(bar, parity, &sm.abort, p.wait_ns)) return true;
+  *reinterpret_cast<volatile int*>(&sm.abort) = 1;
+  set_status(p.status, PISA_DEVERR_WAIT_TIMEOUT);
+  return false;
+}
+
+// Fills the selection bitmap of query block `qi` (validating entries) — all threads of the CTA.
+__device__ void build_bits(uint32_t* bits, const Params& p, int bh, int qi) {
+  if (p.dense) {
+    for (int w = threadIdx.x; w < kWords; w += kThreads) {
+      const int lo = w * 32;
+      bits[w] = lo >= p.nb ? 0u : (p.nb - lo >= 32 ? 0xffffffffu : ((1u << (p.nb - lo)) - 1u));
+    }
+    return;
+  }
+  const int32_t* row = p.sel + ((size_t)bh * p.nb + qi) * p.keep_k;
+  for (int e = threadIdx.x; e < p.keep_k; e += kThreads) {
+    const int j = row[e];
+    bool ok = j >= 0 && j < p.nb;
+    if (e > 0 && row[e - 1] >= j) set_status(p.status, PISA_DEVERR_BAD_SELECTION);
+    if (!ok) {
+      set_status(p.status, PISA_DEVERR_BAD_SELECTION);
+      continue;
+    }
+    const uint32_t old = atomicOr(&bits[j >> 5], 1u << (j & 31));
+    if (old & (1u << (j & 31))) set_status(p.status, PISA_DEVERR_BAD_SELECTION);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, bh = blockIdx.y;
+  const bool pair = p.block == 64;
+
+  // ---- query blocks of this tile ----
+  int qa, qb;
+  bool has_b = false;
+  if (pair) {
+    const int ia = 2 * tile, ib = 2 * tile + 1;
+    qa = p.order ? p.order[(size_t)bh * p.nb + ia] : ia;
+    has_b = ib < p.nb;
+    qb = has_b ? (p.order ? p.order[(size_t)bh * p.nb + ib] : ib) : qa;
+  } else {
+    qa = qb = tile;
+  }
+  if (qa < 0 || qa >= p.nb || qb < 0 || qb >= p.nb) {
+    if (threadIdx.x == 0) set_status(p.status, PISA_DEVERR_BAD_SELECTION);
+    return;
+  }
+
+  // ---- set-up: barriers, TMEM, selection bitmaps ----
+  for (int w = threadIdx.x; w < kWords; w += kThreads) { sm.bitsA[w] = 0u; sm.bitsB[w] = 0u; }
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_q, 1);
+    mbar_init(&sm.bar_kfull, 1);
+    mbar_init(&sm.bar_kempty, 1);
+    mbar_init(&sm.bar_vfull, 1);
+    mbar_init(&sm.bar_vempty, 1);
+    mbar_init(&sm.bar_sfull, 1);
+    mbar_init(&sm.bar_pfull, 128);
+    mbar_init(&sm.bar_odone, 1);
+    mbar_init(&sm.bar_final, 1);
+    mbar_init(&sm.bar_drain, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  build_bits(sm.bitsA, p, bh, qa);
+  if (has_b) build_bits(sm.bitsB, p, bh, qb);
+  __syncthreads();
+  if (!has_b)
+    for (int w = threadIdx.x; w < kWords; w += kThreads) sm.bitsB[w] = sm.bitsA[w];
+  if (warp == 0) {
+    int cnt = 0;
+    for (int w = lane; w < kWords; w += 32) cnt += __popc(sm.bitsA[w] | sm.bitsB[w]);
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) {
+      sm.n_exact = pair ? (cnt + 1) / 2 : cnt;
+      const bool approx = p.mode == PISA_MODE_PISA && !p.dense && p.keep_k < p.nb;
+      sm.n_cent = approx ? (p.nb + 127) / 128 : 0;
+      sm.need_corr = approx ? 1 : 0;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int n_exact = sm.n_exact, T = sm.n_exact + sm.n_cent;
+  const bool need_corr = sm.need_corr != 0;
+
+  if (warp == 4) {
+    // =============================== TMA producer ===============================
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      mbar_expect_tx(&sm.bar_q, kTileBytes);
+      tma_load_3d(sm.q, &maps.q, &sm.bar_q, 0, qa * p.block, bh);
+      tma_load_3d(sm.q + kHalf, &maps.q, &sm.bar_q, 64, qa * p.block, bh);
+      if (pair) {
+        tma_load_3d(sm.q + 64 * 128, &maps.q, &sm.bar_q, 0, qb * p.block, bh);
+        tma_load_3d(sm.q + kHalf + 64 * 128, &maps.q, &sm.bar_q, 64, qb * p.block, bh);
+      }
+      UnionIter it;
+      int issued_k = 0, issued_v = 0;
+      bool ok = true;
+      for (int t = 0; t < T && ok; ++t) {
+        if (t > 0 && !(ok = wait_or_abort(sm, &sm.bar_kempty, (t - 1) & 1, p))) break;
+        const KeyTile kt = key_tile(t, n_exact, pair, it, sm.bitsA, sm.bitsB);
+        const int j1 = kt.j1 >= 0 ? kt.j1 : kt.j0;     // absent second block: reload the first, masked
+        mbar_expect_tx(&sm.bar_kfull, kTileBytes);
+        if (kt.kind == 0) {
+          if (pair) {
+            tma_load_3d(sm.k, &maps.k, &sm.bar_kfull, 0, kt.j0 * 64, bh);
+            tma_load_3d(sm.k + kHalf, &maps.k, &sm.bar_kfull, 64, kt.j0 * 64, bh);
+            tma_load_3d(sm.k + 64 * 128, &maps.k, &sm.bar_kfull, 0, j1 * 64, bh);
+            tma_load_3d(sm.k + kHalf + 64 * 128, &maps.k, &sm.bar_kfull, 64, j1 * 64, bh);
+          } else {
+            tma_load_3d(sm.k, &maps.k, &sm.bar_kfull, 0, kt.j0 * 128, bh);
+            tma_load_3d(sm.k + kHalf, &maps.k, &sm.bar_kfull, 64, kt.j0 * 128, bh);
+          }
+        } else {
+          tma_load_3d(sm.k, &maps.kbar, &sm.bar_kfull, 0, kt.j0, bh);
+          tma_load_3d(sm.k + kHalf, &maps.kbar, &sm.bar_kfull, 64, kt.j0, bh);
+        }
+        ++issued_k;
+        if (t > 0 && !(ok = wait_or_abort(sm, &sm.bar_vempty, (t - 1) & 1, p))) break;
+        mbar_expect_tx(&sm.bar_vfull, kTileBytes);
+        if (kt.kind == 0) {
+          if (pair) {
+            tma_load_3d(sm.v, &maps.v, &sm.bar_vfull, 0, kt.j0 * 64, bh);
+            tma_load_3d(sm.v + kHalf, &maps.v, &sm.bar_vfull, 64, kt.j0 * 64, bh);
+            tma_load_3d(sm.v + 64 * 128, &maps.v, &sm.bar_vfull, 0, j1 * 64, bh);
+            tma_load_3d(sm.v + kHalf + 64 * 128, &maps.v, &sm.bar_vfull, 64, j1 * 64, bh);
+          } else {
+            tma_load_3d(sm.v, &maps.v, &sm.bar_vfull, 0, kt.j0 * 128, bh);
+            tma_load_3d(sm.v + kHalf, &maps.v, &sm.bar_vfull, 64, kt.j0 * 128, bh);
+          }
+        } else {
+          tma_load_3d(sm.v, &maps.vsum, &sm.bar_vfull, 0, kt.j0, bh);
+          tma_load_3d(sm.v + kHalf, &maps.vsum, &sm.bar_vfull, 64, kt.j0, bh);
+        }
+        ++issued_v;
+      }
+      if (ok && need_corr) {
+        if ((ok = wait_or_abort(sm, &sm.bar_kempty, (T - 1) & 1, p))) {
+          mbar_expect_tx(&sm.bar_kfull, kTileBytes);
+          tma_load_3d(sm.k, &maps.hbar, &sm.bar_kfull, 0, 0, bh);
+          tma_load_3d(sm.k + kHalf, &maps.hbar, &sm.bar_kfull, 64, 0, bh);
+          ++issued_k;
+        }
+      }
+      if (!ok) {
+        // drain: every copy issued so far must land before this CTA's shared memory is released
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
+        while (issued_k > 0 && !mbar_try_wait(&sm.bar_kfull, (issued_k - 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+        while (issued_v > 0 && !mbar_try_wait(&sm.bar_vfull, (issued_v - 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+      }
+    }
+  } else if (warp == 5) {
+    // =============================== MMA issuer ===============================
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      const uint32_t q_addr = smem_u32(sm.q), k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+      bool ok = wait_or_abort(sm, &sm.bar_q, 0, p);
+      tc_fence_after();
+      for (int t = 0; t < T && ok; ++t) {
+        if (!(ok = wait_or_abort(sm, &sm.bar_kfull, t & 1, p))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tmem + kColS, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+                 idesc_s, kk > 0);
+        }
+        mma_commit(&sm.bar_kempty);
+        mma_commit(&sm.bar_sfull);
+        if (!(ok = wait_or_abort(sm, &sm.bar_pfull, t & 1, p))) break;
+        if (!(ok = wait_or_abort(sm, &sm.bar_vfull, t & 1, p))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          mma_ts(tmem + kColO, tmem + kColS + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024), idesc_pv,
+                 (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&sm.bar_vempty);
+        mma_commit(&sm.bar_odone);
+      }
+      if (ok && need_corr) {
+        if ((ok = wait_or_abort(sm, &sm.bar_kfull, T & 1, p))) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+            mma_ss(tmem + kColS, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+                   idesc_s, kk > 0);
+          }
+        }
+      }
+      mma_commit(&sm.bar_final);
+      // every MMA issued above has completed once bar_drain flips (bounded)
+      mma_commit(&sm.bar_drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&sm.bar_drain, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
+    }
+  } else {
+    // =========================== softmax + epilogue ===========================
+    // Thread r owns tile row r (TMEM lane r).  Decisions that guard .sync.aligned TMEM accesses are
+    // made warp-uniform.
+    const unsigned FULL = 0xffffffffu;
+    const int r = threadIdx.x;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const bool upper = pair && r >= 64;
+    const uint32_t* bits = upper ? sm.bitsB : sm.bitsA;
+    const int myq = upper ? qb : qa;
+    const int rloc = pair ? (r & 63) : r;
+    const bool row_valid = rloc < block_count(myq, p.L, p.block) && (!upper || has_b);
+    const float last_cnt = (float)block_count(p.nb - 1, p.L, p.block);
+    float m = -INFINITY, l = 0.f, A = 0.f;
+    UnionIter it;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_sfull, t & 1, p));
+      if (!ok) break;
+      tc_fence_after();
+      const KeyTile kt = key_tile(t, n_exact, pair, it, sm.bitsA, sm.bitsB);
+      const bool centroid = kt.kind == 1;
+      float s[128];
+      tmem_ld32(trow + kColS + 0, s);
+      tmem_ld32(trow + kColS + 32, s + 32);
+      tmem_ld32(trow + kColS + 64, s + 64);
+      tmem_ld32(trow + kColS + 96, s + 96);
+      // column validity, 32 columns per word
+      uint32_t vmask[4];
+      if (!centroid) {
+        const int jh1 = pair ? kt.j1 : kt.j0;
+        const bool ok0 = kt.j0 >= 0 && bit_of(bits, kt.j0);
+        const bool ok1 = jh1 >= 0 && bit_of(bits, jh1);
+        const int c0 = ok0 ? block_count(kt.j0, p.L, p.block) : 0;
+        const int c1 = ok1 ? block_count(jh1, p.L, p.block) : 0;
+        if (pair) {
+          vmask[0] = c0 >= 32 ? FULL : ((1u << c0) - 1u);
+          vmask[1] = c0 >= 64 ? FULL : (c0 > 32 ? ((1u << (c0 - 32)) - 1u) : 0u);
+          vmask[2] = c1 >= 32 ? FULL : ((1u << c1) - 1u);
+          vmask[3] = c1 >= 64 ? FULL : (c1 > 32 ? ((1u << (c1 - 32)) - 1u) : 0u);
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int rem = c0 - 32 * g;
+            vmask[g] = rem >= 32 ? FULL : (rem > 0 ? ((1u << rem) - 1u) : 0u);
+          }
+        }
+      } else {
+        const int w0 = kt.j0 >> 5;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int rem = p.nb - (kt.j0 + 32 * g);
+          const uint32_t inr = rem >= 32 ? FULL : (rem > 0 ? ((1u << rem) - 1u) : 0u);
+          vmask[g] = inr & ~(w0 + g < kWords ? bits[w0 + g] : 0u);
+        }
+      }
+      tmem_ld_wait();
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const bool valid = (vmask[c >> 5] >> (c & 31)) & 1u;
+        s[c] = valid ? s[c] * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, s[c]);
+      }
+      const float m_new = fmaxf(m, tmax);
+      const bool grow = m_new > m + 8.f;
+      if (__any_sync(FULL, grow)) {
+        const float f = grow ? ex2(m - m_new) : 1.f;     // ex2(-inf) = 0 on the first valid tile
+        if (t > 0) {
+          // O holds the PV products of earlier tiles: wait for the last one, rescale it in TMEM
+          ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_odone, (t - 1) & 1, p));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            float ov[32];
+            tmem_ld32(trow + kColO + 32 * ch, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ov[x] *= f;
+            tmem_st32(trow + kColO + 32 * ch, ov);
+          }
+          tmem_st_wait();
+        }
+        if (grow) {
+          l *= f;
+          A *= f;
+          m = m_new;
+        }
+      }
+      // P = exp2(s - m) as bf16 pairs, written over the first 64 columns of S in 32-column chunks
+      // (every S value is already in registers)
+      float ls = 0.f, as = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const int c = 32 * ch + x;
+          const float p0 = s[c] == -INFINITY ? 0.f : ex2(s[c] - m);
+          const float p1 = s[c + 1] == -INFINITY ? 0.f : ex2(s[c + 1] - m);
+          if (centroid) {
+            const int jc = kt.j0 + c;
+            const float w0 = jc == p.nb - 1 ? last_cnt : (float)p.block;
+            const float w1 = jc + 1 == p.nb - 1 ? last_cnt : (float)p.block;
+            ls = fmaf(w0, p0, fmaf(w1, p1, ls));
+            as += p0 + p1;
+          } else {
+            ls += p0 + p1;
+          }
+          pk[x >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(trow + kColS + 16 * ch, pk);
+      }
+      l += ls;
+      A += as;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_pfull);
+    }
+    if (ok) ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_final, 0, p));
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.L + (size_t)myq * p.block + rloc) * D;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        float ov[32], cv[32];
+        tmem_ld32(trow + kColO + 32 * ch, ov);
+        if (need_corr) tmem_ld32(trow + kColS + 32 * ch, cv);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          float a = ov[x], b = ov[x + 1];
+          if (need_corr) {
+            a = fmaf(A, cv[x], a);
+            b = fmaf(A, cv[x + 1], b);
+          }
+          pk[x >> 1] = pack_bf16x2(a * inv, b * inv);
+        }
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * ch);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  __syncwarp();
+  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+size_t attention_sm100_smem_bytes() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
+                                   int keep_k, int mode, void* o, int* status, unsigned long long wait_ns,
+                                   cudaStream_t stream) {
+  Params p;
+  p.L = g.L;
+  p.nb = g.nb;
+  p.block = g.block;
+  p.keep_k = keep_k;
+  p.mode = mode;
+  p.dense = keep_k == g.nb;
+  p.scale_log2 = g.scale * 1.4426950408889634f;
+  p.sel = sel;
+  p.order = order;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.status = status;
+  p.wait_ns = wait_ns;
+  const size_t smem = attention_sm100_smem_bytes();
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(attn_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+  const int ntiles = g.block == 64 ? (g.nb + 1) / 2 : g.nb;
+  attn_sm100<<<dim3(ntiles, g.BH()), kThreads, smem, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+}  // namespace pisa

@@ -1,6 +1,7 @@
 // Shared device/host definitions of the PISA library (internal; not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -45,11 +46,26 @@ __device__ __forceinline__ int block_count(int j, int L, int block) {
   return e - s;
 }
 
+// TMA descriptors of one pisa_attention call (bf16 path).
+struct AttnMaps {
+  CUtensorMap q, k, v, kbar, vsum, hbar;
+};
+
+// Encodes a 3-D bf16 tensor [batch][rows][inner] (row-major) with a {64, box_rows, 1} box and
+// 128-byte swizzling; false if the driver entry point is unavailable or rejects the arguments.
+bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                    uint32_t box_rows);
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits: 2 s
+
 // ---- launchers (defined in the kernel translation units) ----
 cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,
                                    const pisa_stats& st, void* ws, cudaStream_t stream);
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream);
+cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
+                                   int keep_k, int mode, void* o, int* status, unsigned long long wait_ns,
+                                   cudaStream_t stream);
 cudaError_t launch_attention_simt(const Dims& g, const void* q, const void* k, const void* v,
                                   const pisa_stats& st, const int32_t* sel, int keep_k, int mode,
                                   void* o, int* status, cudaStream_t stream);

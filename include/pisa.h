@@ -67,7 +67,7 @@ typedef struct {
   int32_t head_dim;       /* d */
   int32_t block;          /* tokens per key block and per query block */
   int32_t dtype;          /* pisa_dtype of q, k, v, o */
-  float   softmax_scale;  /* s: multiplies every logit and the first-order correction */
+  float   softmax_scale;  /* s > 0: multiplies every logit and the first-order correction */
 } pisa_shape;
 
 /* Per-head block statistics written by pisa_precompute.  nb = pisa_num_blocks(L, block).

@@ -18,7 +18,7 @@ pisa_status check_shape(const pisa_shape* s, Dims* g) {
   if (s->batch < 1 || s->heads < 1 || s->seq_len < 1 || s->head_dim < 1 || s->block < 1)
     return PISA_ERR_INVALID_ARG;
   if (s->dtype != PISA_BF16 && s->dtype != PISA_FP32) return PISA_ERR_INVALID_ARG;
-  if (!std::isfinite(s->softmax_scale)) return PISA_ERR_INVALID_ARG;
+  if (!std::isfinite(s->softmax_scale) || !(s->softmax_scale > 0.f)) return PISA_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
   if (s->dtype == PISA_BF16 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
   if (s->block != 64 && s->block != 128) return PISA_ERR_UNSUPPORTED;
@@ -135,7 +135,9 @@ pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* 
     return PISA_ERR_INVALID_ARG;
   if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
   if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
-  return cuda_status(launch_precompute_simt(g, q, k, v, *stats, ws, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (g.dtype == PISA_BF16) return cuda_status(launch_precompute_sm100(g, q, k, v, *stats, ws, cs));
+  return cuda_status(launch_precompute_simt(g, q, k, v, *stats, ws, cs));
 }
 
 pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,

@@ -378,68 +378,78 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         }
       }
       tmem_ld_wait();
-      float tmax = -INFINITY;
+      // masks touch only 32-column groups that are partly invalid (warp-uniform: a warp's 32 rows
+      // belong to one query block)
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const bool valid = (vmask[c >> 5] >> (c & 31)) & 1u;
-        s[c] = valid ? s[c] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, s[c]);
-      }
-      const float m_new = fmaxf(m, tmax);
-      const bool grow = m_new > m + kRescaleLog2;
-      if (__any_sync(FULL, grow)) {
-        const float f = grow ? ex2(m - m_new) : 1.f;     // ex2(-inf) = 0 on the first valid tile
-        if (t > 0) {
-          // O holds the PV products of earlier tiles: wait for the last one, rescale it in TMEM
-          ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_odone, (t - 1) & 1, p));
-          if (!ok) break;
-          tc_fence_after();
+      for (int g = 0; g < 4; ++g) {
+        const uint32_t vm = vmask[g];
+        if (vm != FULL) {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            float ov[32];
-            tmem_ld32(trow + kColO + 32 * ch, ov);
-            tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) ov[x] *= f;
-            tmem_st32(trow + kColO + 32 * ch, ov);
-          }
-          tmem_st_wait();
-        }
-        if (grow) {
-          l *= f;
-          A *= f;
-          m = m_new;
+          for (int x = 0; x < 32; ++x) s[32 * g + x] = ((vm >> x) & 1u) ? s[32 * g + x] : -INFINITY;
         }
       }
-      // P = exp2(s - m) as bf16 pairs, written over the first 64 columns of S in 32-column chunks
-      // (every S value is already in registers).  The denominator and A sum the same bf16-rounded
-      // values the PV product uses, so a row dominated by one key keeps o = v exactly.
-      float ls = 0.f, as = 0.f;
+      float t0 = s[0], t1 = s[1], t2 = s[2], t3 = s[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        t0 = fmaxf(t0, s[c]);
+        t1 = fmaxf(t1, s[c + 1]);
+        t2 = fmaxf(t2, s[c + 2]);
+        t3 = fmaxf(t3, s[c + 3]);
+      }
+      const float m_new = fmaxf(m, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));   // raw logit units
+      const bool grow = m_new > m;
+      const float f = grow ? ex2((m - m_new) * p.scale_log2) : 1.f;   // 0 when m = -inf
+      if (grow) {
+        l *= f;
+        A *= f;
+        m = m_new;
+      }
+      float slast = -INFINITY;     // raw logit of the last (short) key block, when this tile holds it
+      const int cl = p.nb - 1 - kt.j0;
+      const bool has_last = centroid && cl >= 0 && cl < 128 && last_cnt != (float)p.block;
+      if (has_last) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) slast = c == cl ? s[c] : slast;
+      }
+      // p = 2^(s*scale*log2e - m*scale*log2e); masked entries are -inf and give exactly 0
+      const float mb = m == -INFINITY ? 0.f : m * p.scale_log2;
+      float ls = 0.f;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          const int c = 32 * ch + x;
-          const uint32_t pp = pack_bf16x2(s[c] == -INFINITY ? 0.f : ex2(s[c] - m),
-                                          s[c + 1] == -INFINITY ? 0.f : ex2(s[c + 1] - m));
-          const float p0 = __uint_as_float(pp << 16);
-          const float p1 = __uint_as_float(pp & 0xffff0000u);
-          if (centroid) {
-            const int jc = kt.j0 + c;
-            const float w0 = jc == p.nb - 1 ? last_cnt : (float)p.block;
-            const float w1 = jc + 1 == p.nb - 1 ? last_cnt : (float)p.block;
-            ls = fmaf(w0, p0, fmaf(w1, p1, ls));
-            as += p0 + p1;
-          } else {
-            ls += p0 + p1;
-          }
-          pk[x >> 1] = pp;
+          const float p0 = ex2(fmaf(s[32 * ch + x], p.scale_log2, -mb));
+          const float p1 = ex2(fmaf(s[32 * ch + x + 1], p.scale_log2, -mb));
+          ls += p0 + p1;
+          pk[x >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st16(trow + kColS + 16 * ch, pk);
       }
-      l += ls;
-      A += as;
+      if (centroid) {
+        // alpha of every unselected block enters D with weight cnt_j: `block` except the last one
+        A += ls;
+        l = fmaf((float)p.block, ls, l);
+        if (has_last) l = fmaf(last_cnt - (float)p.block, ex2(fmaf(slast, p.scale_log2, -mb)), l);
+      } else {
+        l += ls;
+      }
+      // O holds the PV products of earlier tiles (already complete: S(t) was committed after
+      // PV(t-1)); rescale it before PV(t) is released
+      if (__any_sync(FULL, grow) && t > 0) {
+        ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_odone, (t - 1) & 1, p));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          float ov[32];
+          tmem_ld32(trow + kColO + 32 * ch, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ov[x] *= f;
+          tmem_st32(trow + kColO + 32 * ch, ov);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&sm.bar_pfull);

@@ -61,6 +61,10 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier
 // ---- launchers (defined in the kernel translation units) ----
 cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,
                                    const pisa_stats& st, void* ws, cudaStream_t stream);
+cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v,
+                                    const pisa_stats& st, void* ws, cudaStream_t stream);
+cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const pisa_stats& st,
+                               cudaStream_t stream);
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream);
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,

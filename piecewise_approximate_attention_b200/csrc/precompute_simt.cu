@@ -179,6 +179,18 @@ cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, cons
 
 }  // namespace
 
+cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const pisa_stats& st,
+                               cudaStream_t stream) {
+  dim3 grid((g.d * g.d + kThreads - 1) / kThreads, g.BH());
+  if (g.d == 64)
+    hbar_reduce<64><<<grid, kThreads, 0, stream>>>(partials, nparts, g.nb, g.scale, st.hbar,
+                                                   static_cast<__nv_bfloat16*>(st.hbar_op));
+  else
+    hbar_reduce<128><<<grid, kThreads, 0, stream>>>(partials, nparts, g.nb, g.scale, st.hbar,
+                                                    static_cast<__nv_bfloat16*>(st.hbar_op));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,
                                    const pisa_stats& st, void* ws, cudaStream_t stream) {
   if (g.dtype == PISA_FP32) {

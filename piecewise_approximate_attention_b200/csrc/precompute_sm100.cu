@@ -1,0 +1,442 @@
+// Block statistics on sm_100a for bf16 inputs: TMA tiles, tcgen05 contractions for H_j.
+//
+// "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion Transformers", §2 방법론:
+// the pre-computation step (하드웨어 구현 step 1) produces block centroids kbar_j and value sums
+// (zeroth-order term), the global statistic Hbar = mean_j H_j with H_j = sum_n (k_n - kbar_j)^T v_n
+// (first-order correction) and, for covariance-aware routing (공분산 인식 라우팅),
+// M_j = ||H_j - Hbar||_F.  Query-block means qbar_i are produced in the same pass for routing.
+//
+// Pass A (one CTA per head and group of kBlocksPerPart key blocks): streams 128-row tiles of Q, K, V
+// with TMA, reduces block column sums on CUDA cores straight from the swizzled tiles, and
+// accumulates sum_n k_n v_n^T over the whole group in TMEM with tcgen05 (both operands MN-major,
+// fp32 accumulate).  Its epilogue subtracts sum_j kbar_j vsum_j^T, giving the group's partial
+// sum_j H_j.  The fixed-order reduction of the partials (hbar_reduce) gives Hbar.
+// Pass B (one CTA per head and group of key blocks): re-streams K, V, recomputes each H_j with one
+// MMA chain per block into double-buffered TMEM and reduces ||H_j - kbar_j vsum_j^T - Hbar||^2 in
+// the epilogue.  Re-reading K, V (2 L d bf16) costs less HBM traffic than storing and re-reading
+// H_j (nb d^2 fp32).
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace pisa {
+namespace {
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int kThreads = 192;
+constexpr int kHalf = 128 * 64 * 2;      // 128 rows x 64 columns of bf16: 16 KB
+constexpr int kTile = 2 * kHalf;         // 128 x 128 bf16 tile: 32 KB
+constexpr uint32_t kIdescKV = idesc_bf16_f32(128, 128, true, true);   // D[a][c] += sum_n K[n][a] V[n][c]
+
+__device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Every epilogue thread reaches this after a bounded wait; the OR-reduction at the barrier gives all 128
+// threads the same answer, so no later named barrier can strand a warp.
+__device__ __forceinline__ bool epi_any_failed(bool failed) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, 1, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)failed)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, int* abort, int* status,
+                                         unsigned long long ns) {
+  if (mbar_wait_bounded(bar, parity, abort, ns)) return true;
+  *reinterpret_cast<volatile int*>(abort) = 1;
+  set_status(status, PISA_DEVERR_WAIT_TIMEOUT);
+  return false;
+}
+
+// Sums of 8 consecutive columns (chunk cc of 16) over the rows r in [r0, r1) with r = rg (mod 8), read
+// from a 128B-swizzled [128 x 128] bf16 tile.  r0 is a multiple of 8.
+__device__ __forceinline__ void colsum8(const uint8_t* tile, int cc, int rg, int r0, int r1, float acc[8]) {
+  const uint8_t* base = tile + (cc >> 3) * kHalf + (((cc & 7) ^ rg) << 4);
+#pragma unroll 4
+  for (int r = r0 + rg; r < r1; r += 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(base + r * 128);
+    acc[0] += __uint_as_float(u.x << 16);
+    acc[1] += __uint_as_float(u.x & 0xffff0000u);
+    acc[2] += __uint_as_float(u.y << 16);
+    acc[3] += __uint_as_float(u.y & 0xffff0000u);
+    acc[4] += __uint_as_float(u.z << 16);
+    acc[5] += __uint_as_float(u.z & 0xffff0000u);
+    acc[6] += __uint_as_float(u.w << 16);
+    acc[7] += __uint_as_float(u.w & 0xffff0000u);
+  }
+}
+
+struct KVMaps {
+  CUtensorMap q, k, v;     // [BH][L][128] bf16, box {64, 128, 1}
+};
+
+struct PreParams {
+  int L, nb, block;
+  pisa_stats st;
+  float* partials;
+  int* status;
+  unsigned long long wait_ns;
+};
+
+// ----------------------------------------------------------------------------------------------
+// Pass A
+// ----------------------------------------------------------------------------------------------
+struct alignas(1024) SmemA {
+  uint8_t q[2][kTile];
+  uint8_t k[2][kTile];
+  uint8_t v[2][kTile];
+  float red[3][8][128];
+  float ck[2][128], cv[2][128];
+  uint64_t full[2], empty[2], acc_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_constant__ KVMaps maps, const PreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemA& sm = *reinterpret_cast<SmemA*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int part = blockIdx.x, bh = blockIdx.y, nparts = gridDim.x;
+  const int jb0 = part * kBlocksPerPart, jb1 = min(p.nb, jb0 + kBlocksPerPart);
+  const int row0 = jb0 * p.block, row1 = min(p.L, jb1 * p.block);
+  const int ntile = (row1 - row0 + 127) / 128;
+  const int bpt = 128 / p.block;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 129);
+    }
+    mbar_init(&sm.acc_done, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&sm.tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int t = 0; t < ntile; ++t) {
+        const int s = t & 1;
+        if (t >= 2 && !(ok = wait_bar(&sm.empty[s], ((t >> 1) - 1) & 1, &sm.abort, p.status, p.wait_ns))) break;
+        const int y = row0 + t * 128;
+        mbar_expect_tx(&sm.full[s], 3 * kTile);
+        tma_load_3d(sm.q[s], &maps.q, &sm.full[s], 0, y, bh);
+        tma_load_3d(sm.q[s] + kHalf, &maps.q, &sm.full[s], 64, y, bh);
+        tma_load_3d(sm.k[s], &maps.k, &sm.full[s], 0, y, bh);
+        tma_load_3d(sm.k[s] + kHalf, &maps.k, &sm.full[s], 64, y, bh);
+        tma_load_3d(sm.v[s], &maps.v, &sm.full[s], 0, y, bh);
+        tma_load_3d(sm.v[s] + kHalf, &maps.v, &sm.full[s], 64, y, bh);
+        ++issued;
+      }
+      if (!ok) {   // let issued copies land before shared memory is released
+        const uint64_t t0 = globaltimer_ns();
+        for (int t = max(0, issued - 2); t < issued; ++t)
+          while (!mbar_try_wait(&sm.full[t & 1], (t >> 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      bool ok = true;
+      for (int t = 0; t < ntile && ok; ++t) {
+        const int s = t & 1;
+        if (!(ok = wait_bar(&sm.full[s], (t >> 1) & 1, &sm.abort, p.status, p.wait_ns))) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sm.k[s]), va = smem_u32(sm.v[s]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem, smem_desc_sw128(ka + kk * 2048, kHalf, 1024), smem_desc_sw128(va + kk * 2048, kHalf, 1024),
+                 kIdescKV, (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.empty[s]);
+      }
+      mma_commit(&sm.acc_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&sm.acc_done, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
+    }
+  } else {
+    // column sums + rank-1 centring terms (threads 0..127)
+    const int tid = threadIdx.x, cc = tid & 15, rg = tid >> 4;
+    float corr[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) corr[c] = 0.f;
+    bool ok = true;
+    int nblk = 0;
+    for (int t = 0; t < ntile; ++t) {
+      const int s = t & 1;
+      ok = !epi_any_failed(!wait_bar(&sm.full[s], (t >> 1) & 1, &sm.abort, p.status, p.wait_ns));
+      if (!ok) break;
+      for (int b = 0; b < bpt; ++b) {
+        const int j = jb0 + t * bpt + b;
+        if (j >= jb1) break;
+        const int cnt = block_count(j, p.L, p.block);
+        const int r0 = b * p.block;
+        float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0}, av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        colsum8(sm.q[s], cc, rg, r0, r0 + cnt, aq);
+        colsum8(sm.k[s], cc, rg, r0, r0 + cnt, ak);
+        colsum8(sm.v[s], cc, rg, r0, r0 + cnt, av);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          sm.red[0][rg][cc * 8 + x] = aq[x];
+          sm.red[1][rg][cc * 8 + x] = ak[x];
+          sm.red[2][rg][cc * 8 + x] = av[x];
+        }
+        bar_epi();
+        const int c = tid;
+        float sq = 0.f, sk = 0.f, sv = 0.f;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          sq += sm.red[0][g][c];
+          sk += sm.red[1][g][c];
+          sv += sm.red[2][g][c];
+        }
+        const float inv = 1.f / (float)cnt;
+        const size_t so = ((size_t)bh * p.nb + j) * D + c;
+        p.st.qbar[so] = sq * inv;
+        p.st.kbar[so] = sk * inv;
+        p.st.vsum[so] = sv;
+        reinterpret_cast<__nv_bfloat16*>(p.st.kbar_op)[so] = __float2bfloat16_rn(sk * inv);
+        reinterpret_cast<__nv_bfloat16*>(p.st.vsum_op)[so] = __float2bfloat16_rn(sv);
+        const int pb = nblk & 1;
+        sm.ck[pb][c] = sk * inv;
+        sm.cv[pb][c] = sv;
+        bar_epi();
+        const float ka = sm.ck[pb][tid];
+#pragma unroll
+        for (int x = 0; x < D; ++x) corr[x] = fmaf(ka, sm.cv[pb][x], corr[x]);
+        ++nblk;
+      }
+      mbar_arrive(&sm.empty[s]);
+    }
+    if (ok) ok = !epi_any_failed(!wait_bar(&sm.acc_done, 0, &sm.abort, p.status, p.wait_ns));
+    if (ok) {
+      tc_fence_after();
+      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+      float* out = p.partials + ((size_t)bh * nparts + part) * D * D + (size_t)tid * D;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        float a[32];
+        tmem_ld32(trow + 32 * ch, a);
+        tmem_ld_wait();
+        if (ntile == 0) {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) a[x] = 0.f;
+        }
+#pragma unroll
+        for (int x = 0; x < 32; x += 4)
+          *reinterpret_cast<float4*>(out + 32 * ch + x) =
+              make_float4(a[x] - corr[32 * ch + x], a[x + 1] - corr[32 * ch + x + 1], a[x + 2] - corr[32 * ch + x + 2],
+                          a[x + 3] - corr[32 * ch + x + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ----------------------------------------------------------------------------------------------
+// Pass B
+// ----------------------------------------------------------------------------------------------
+constexpr int kStagesB = 3;
+constexpr int kBlocksPerCtaB = 16;
+
+struct alignas(1024) SmemB {
+  uint8_t k[kStagesB][kTile];
+  uint8_t v[kStagesB][kTile];
+  float vs[2][2][128];
+  float red[2][4];
+  uint64_t full[kStagesB], empty[kStagesB], acc_full[2], acc_empty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_constant__ KVMaps maps, const PreParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemB& sm = *reinterpret_cast<SmemB*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = blockIdx.x, bh = blockIdx.y;
+  const int jb0 = grp * kBlocksPerCtaB, jb1 = min(p.nb, jb0 + kBlocksPerCtaB);
+  const int row0 = jb0 * p.block, row1 = min(p.L, jb1 * p.block);
+  const int ntile = (row1 - row0 + 127) / 128;
+  const int bpt = 128 / p.block;
+  const int ksteps = p.block / 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStagesB; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.acc_full[b], 1);
+      mbar_init(&sm.acc_empty[b], 128);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int t = 0; t < ntile; ++t) {
+        const int s = t % kStagesB;
+        if (t >= kStagesB &&
+            !(ok = wait_bar(&sm.empty[s], ((t / kStagesB) - 1) & 1, &sm.abort, p.status, p.wait_ns)))
+          break;
+        const int y = row0 + t * 128;
+        mbar_expect_tx(&sm.full[s], 2 * kTile);
+        tma_load_3d(sm.k[s], &maps.k, &sm.full[s], 0, y, bh);
+        tma_load_3d(sm.k[s] + kHalf, &maps.k, &sm.full[s], 64, y, bh);
+        tma_load_3d(sm.v[s], &maps.v, &sm.full[s], 0, y, bh);
+        tma_load_3d(sm.v[s] + kHalf, &maps.v, &sm.full[s], 64, y, bh);
+        ++issued;
+      }
+      if (!ok) {
+        const uint64_t t0 = globaltimer_ns();
+        for (int t = max(0, issued - kStagesB); t < issued; ++t)
+          while (!mbar_try_wait(&sm.full[t % kStagesB], (t / kStagesB) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      bool ok = true;
+      for (int t = 0; t < ntile && ok; ++t) {
+        const int s = t % kStagesB, buf = t & 1;
+        if (!(ok = wait_bar(&sm.full[s], (t / kStagesB) & 1, &sm.abort, p.status, p.wait_ns))) break;
+        if (t >= 2 && !(ok = wait_bar(&sm.acc_empty[buf], ((t >> 1) - 1) & 1, &sm.abort, p.status, p.wait_ns))) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sm.k[s]), va = smem_u32(sm.v[s]);
+        for (int b = 0; b < bpt; ++b) {
+          const uint32_t d = tmem + (uint32_t)(buf * 256 + b * 128);
+          for (int kk = 0; kk < ksteps; ++kk) {
+            const uint32_t off = (uint32_t)(b * p.block + kk * 16) * 128;
+            mma_ss(d, smem_desc_sw128(ka + off, kHalf, 1024), smem_desc_sw128(va + off, kHalf, 1024), kIdescKV,
+                   kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(&sm.empty[s]);
+        mma_commit(&sm.acc_full[buf]);
+      }
+      mma_commit(&sm.drain);      // completes once every MMA above has: TMEM may then be released
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
+    }
+  } else {
+    const int a = threadIdx.x;                       // H row a == TMEM lane a
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    float hb[D];
+    const float* hbar = p.st.hbar + (size_t)bh * D * D + (size_t)a * D;
+#pragma unroll
+    for (int x = 0; x < D; x += 4) {
+      const float4 h4 = *reinterpret_cast<const float4*>(hbar + x);
+      hb[x] = h4.x;
+      hb[x + 1] = h4.y;
+      hb[x + 2] = h4.z;
+      hb[x + 3] = h4.w;
+    }
+    bool ok = true;
+    for (int t = 0; t < ntile; ++t) {
+      const int buf = t & 1;
+      ok = !epi_any_failed(!wait_bar(&sm.acc_full[buf], (t >> 1) & 1, &sm.abort, p.status, p.wait_ns));
+      if (!ok) break;
+      tc_fence_after();
+      for (int b = 0; b < bpt; ++b) {
+        const int j = jb0 + t * bpt + b;
+        const bool live = j < jb1;
+        const size_t so = ((size_t)bh * p.nb + (live ? j : 0)) * D;
+        sm.vs[buf][b][a] = live ? p.st.vsum[so + a] : 0.f;
+        const float kb = live ? p.st.kbar[so + a] : 0.f;
+        bar_epi();
+        float ss = 0.f;
+        float* Hout = (live && p.st.H) ? p.st.H + ((size_t)bh * p.nb + j) * D * D + (size_t)a * D : nullptr;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          float h[32];
+          tmem_ld32(trow + (uint32_t)(buf * 256 + b * 128 + 32 * ch), h);
+          tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int c = 32 * ch + x;
+            h[x] = fmaf(-kb, sm.vs[buf][b][c], h[x]);
+            const float dl = h[x] - hb[c];
+            ss = fmaf(dl, dl, ss);
+          }
+          if (Hout) {
+#pragma unroll
+            for (int x = 0; x < 32; x += 4)
+              *reinterpret_cast<float4*>(Hout + 32 * ch + x) = make_float4(h[x], h[x + 1], h[x + 2], h[x + 3]);
+          }
+        }
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) sm.red[b][warp] = ss;
+        bar_epi();
+        if (a == 0 && live) p.st.M[(size_t)bh * p.nb + j] = sqrtf(sm.red[b][0] + sm.red[b][1] + sm.red[b][2] + sm.red[b][3]);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.acc_empty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v, const pisa_stats& st,
+                                    void* ws, cudaStream_t stream) {
+  KVMaps maps;
+  const uint64_t bh = (uint64_t)g.BH();
+  if (!encode_bf16_3d(&maps.q, q, D, g.L, bh, 128) || !encode_bf16_3d(&maps.k, k, D, g.L, bh, 128) ||
+      !encode_bf16_3d(&maps.v, v, D, g.L, bh, 128))
+    return cudaErrorInvalidValue;
+  PreParams p;
+  p.L = g.L;
+  p.nb = g.nb;
+  p.block = g.block;
+  p.st = st;
+  p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
+  p.status = static_cast<int*>(ws);
+  p.wait_ns = kWaitLimitNs;
+  const size_t smem_a = sizeof(SmemA) + 1024, smem_b = sizeof(SmemB) + 1024;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(stats_a_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
+  if ((e = cudaFuncSetAttribute(cov_norm_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
+  const int nparts = num_parts(g);
+  stats_a_sm100<<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(maps, p);
+  if ((e = launch_hbar_reduce(g, p.partials, nparts, st, stream))) return e;
+  cov_norm_sm100<<<dim3((g.nb + kBlocksPerCtaB - 1) / kBlocksPerCtaB, g.BH()), kThreads, smem_b, stream>>>(maps, p);
+  return cudaGetLastError();
+}
+
+}  // namespace pisa

@@ -70,6 +70,8 @@ def test_stats_bytes_and_carve_are_host_only():
     (dict(batch=0), C.PISA_ERR_INVALID_ARG),
     (dict(dtype=7), C.PISA_ERR_INVALID_ARG),
     (dict(softmax_scale=float("nan")), C.PISA_ERR_INVALID_ARG),
+    (dict(softmax_scale=0.0), C.PISA_ERR_INVALID_ARG),
+    (dict(softmax_scale=-1.0), C.PISA_ERR_INVALID_ARG),
     (dict(seq_len=64 * 4097), C.PISA_ERR_UNSUPPORTED),
 ])
 def test_bad_shapes_rejected(kw, expect):

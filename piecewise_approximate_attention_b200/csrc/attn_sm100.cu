@@ -43,7 +43,6 @@ constexpr int kTileBytes = 2 * kHalf;      // 32 KB
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColO = 128;
 constexpr int kWords = 128;                // selection bitmap words (nb <= 4096)
-constexpr float kRescaleLog2 = 0.f;        // rescale O when the row max grows by more than this
 
 struct alignas(1024) Smem {
   uint8_t v[kTileBytes];

@@ -113,6 +113,23 @@ PISA_API size_t pisa_workspace_bytes(const pisa_shape* shape);
 PISA_API pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
                             const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream);
 
+/* pisa_precompute without a caller workspace, for callers that cannot allocate device memory (a
+ * plugin whose host framework owns every device allocation, or a path that must not call cudaMalloc
+ * because it may synchronise the device).  The method's description has no counterpart to this call;
+ * it exists for such callers.  It runs the same kernels as pisa_precompute, with the scratch taken
+ * from a fixed 16 MiB array in the library's device memory, which every device that loads the
+ * library holds until the process exits.  It allocates nothing and frees nothing.
+ *   - Shapes whose pisa_workspace_bytes exceeds 16 MiB return PISA_ERR_UNSUPPORTED and enqueue
+ *     nothing; other invalid arguments are rejected exactly as by pisa_precompute.
+ *   - The first call on a device looks up the array's device address on that device (a host-side
+ *     CUDA runtime query); make that first call before any stream capture.
+ *   - Every call, on any stream, shares the one array: calls that overlap on the GPU race.  Each
+ *     call clears the status word it uses before its kernels start; device-side wait timeouts of
+ *     this call are not reported to the caller.
+ * q, k, v, stats and stream as for pisa_precompute. */
+PISA_API pisa_status pisa_precompute_noalloc(const pisa_shape* shape, const void* q, const void* k,
+                                             const void* v, const pisa_stats* stats, pisa_stream_t stream);
+
 /* Covariance-aware top-k routing (§2 공분산 인식 라우팅):
  *   s_ij = softmax_scale * qbar_i . kbar_j
  *   P_ij = cnt_j exp(s_ij) / sum_l cnt_l exp(s_il)

@@ -19,7 +19,8 @@ PISA_MODE_PISA, PISA_MODE_EXACT_ONLY = 0, 1
 PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
-           "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string")
+           "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string",
+           "pisa_precompute_noalloc")
 
 
 class PisaShape(ctypes.Structure):
@@ -63,6 +64,7 @@ def lib() -> ctypes.CDLL:
             "pisa_attention": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, vp, i32, i32, vp, vp, sz, vp]),
             "pisa_read_device_error": (i32, [vp, P(i32), vp]),
             "pisa_status_string": (ctypes.c_char_p, [i32]),
+            "pisa_precompute_noalloc": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -172,6 +174,12 @@ def alloc_workspace(shape: PisaShape, device):
 def pisa_precompute(shape: PisaShape, q, k, v, stats: Stats, ws, stream=None):
     _check(lib().pisa_precompute(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(stats.c), _ptr(ws),
                                  ws.numel(), _stream(stream)), "pisa_precompute")
+
+
+def pisa_precompute_noalloc(shape: PisaShape, q, k, v, stats: Stats, stream=None):
+    """pisa_precompute with the library's fixed device scratch instead of a caller workspace."""
+    _check(lib().pisa_precompute_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(stats.c),
+                                         _stream(stream)), "pisa_precompute_noalloc")
 
 
 def pisa_route(shape: PisaShape, stats: Stats, keep_k: int, lam: float, sel, order=None, scores=None, stream=None):

@@ -43,12 +43,21 @@ constexpr int kTileBytes = 2 * kHalf;      // 32 KB
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColO = 128;
 constexpr int kWords = 128;                // selection bitmap words (nb <= 4096)
+#ifndef PISA_ATTN_KSTAGES
+#define PISA_ATTN_KSTAGES 1
+#endif
+#ifndef PISA_ATTN_VSTAGES
+#define PISA_ATTN_VSTAGES 1
+#endif
+constexpr int kKS = PISA_ATTN_KSTAGES;     // key-tile buffers in shared memory
+constexpr int kVS = PISA_ATTN_VSTAGES;     // value-tile buffers
 
 struct alignas(1024) Smem {
-  uint8_t v[kTileBytes];
+  uint8_t v[kVS][kTileBytes];
   uint8_t q[kTileBytes];
-  uint8_t k[kTileBytes];
-  uint64_t bar_q, bar_kfull, bar_kempty, bar_vfull, bar_vempty, bar_sfull, bar_pfull, bar_odone, bar_final, bar_drain;
+  uint8_t k[kKS][kTileBytes];
+  uint64_t bar_kfull[kKS], bar_kempty[kKS], bar_vfull[kVS], bar_vempty[kVS];
+  uint64_t bar_q, bar_sfull, bar_pfull, bar_odone, bar_final, bar_drain;
   uint32_t tmem_base;
   int abort;
   int n_exact, n_cent, need_corr;
@@ -163,10 +172,14 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
   for (int w = threadIdx.x; w < kWords; w += kThreads) { sm.bitsA[w] = 0u; sm.bitsB[w] = 0u; }
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
-    mbar_init(&sm.bar_kfull, 1);
-    mbar_init(&sm.bar_kempty, 1);
-    mbar_init(&sm.bar_vfull, 1);
-    mbar_init(&sm.bar_vempty, 1);
+    for (int i = 0; i < kKS; ++i) {
+      mbar_init(&sm.bar_kfull[i], 1);
+      mbar_init(&sm.bar_kempty[i], 1);
+    }
+    for (int i = 0; i < kVS; ++i) {
+      mbar_init(&sm.bar_vfull[i], 1);
+      mbar_init(&sm.bar_vempty[i], 1);
+    }
     mbar_init(&sm.bar_sfull, 1);
     mbar_init(&sm.bar_pfull, 128);
     mbar_init(&sm.bar_odone, 1);
@@ -220,48 +233,54 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       int issued_k = 0, issued_v = 0;
       bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
-        if (t > 0 && !(ok = wait_or_abort(sm, &sm.bar_kempty, (t - 1) & 1, p))) break;
+        const int ks = t % kKS, vs = t % kVS;
+        if (t >= kKS && !(ok = wait_or_abort(sm, &sm.bar_kempty[ks], ((t / kKS) - 1) & 1, p))) break;
         const KeyTile kt = key_tile(t, n_exact, pair, it, sm.bitsA, sm.bitsB);
         const int j1 = kt.j1 >= 0 ? kt.j1 : kt.j0;     // absent second block: reload the first, masked
-        mbar_expect_tx(&sm.bar_kfull, kTileBytes);
+        uint8_t* kb = sm.k[ks];
+        uint64_t* kf = &sm.bar_kfull[ks];
+        mbar_expect_tx(kf, kTileBytes);
         if (kt.kind == 0) {
           if (pair) {
-            tma_load_3d(sm.k, &maps.k, &sm.bar_kfull, 0, kt.j0 * 64, bh);
-            tma_load_3d(sm.k + kHalf, &maps.k, &sm.bar_kfull, 64, kt.j0 * 64, bh);
-            tma_load_3d(sm.k + 64 * 128, &maps.k, &sm.bar_kfull, 0, j1 * 64, bh);
-            tma_load_3d(sm.k + kHalf + 64 * 128, &maps.k, &sm.bar_kfull, 64, j1 * 64, bh);
+            tma_load_3d(kb, &maps.k, kf, 0, kt.j0 * 64, bh);
+            tma_load_3d(kb + kHalf, &maps.k, kf, 64, kt.j0 * 64, bh);
+            tma_load_3d(kb + 64 * 128, &maps.k, kf, 0, j1 * 64, bh);
+            tma_load_3d(kb + kHalf + 64 * 128, &maps.k, kf, 64, j1 * 64, bh);
           } else {
-            tma_load_3d(sm.k, &maps.k, &sm.bar_kfull, 0, kt.j0 * 128, bh);
-            tma_load_3d(sm.k + kHalf, &maps.k, &sm.bar_kfull, 64, kt.j0 * 128, bh);
+            tma_load_3d(kb, &maps.k, kf, 0, kt.j0 * 128, bh);
+            tma_load_3d(kb + kHalf, &maps.k, kf, 64, kt.j0 * 128, bh);
           }
         } else {
-          tma_load_3d(sm.k, &maps.kbar, &sm.bar_kfull, 0, kt.j0, bh);
-          tma_load_3d(sm.k + kHalf, &maps.kbar, &sm.bar_kfull, 64, kt.j0, bh);
+          tma_load_3d(kb, &maps.kbar, kf, 0, kt.j0, bh);
+          tma_load_3d(kb + kHalf, &maps.kbar, kf, 64, kt.j0, bh);
         }
         ++issued_k;
-        if (t > 0 && !(ok = wait_or_abort(sm, &sm.bar_vempty, (t - 1) & 1, p))) break;
-        mbar_expect_tx(&sm.bar_vfull, kTileBytes);
+        if (t >= kVS && !(ok = wait_or_abort(sm, &sm.bar_vempty[vs], ((t / kVS) - 1) & 1, p))) break;
+        uint8_t* vb = sm.v[vs];
+        uint64_t* vf = &sm.bar_vfull[vs];
+        mbar_expect_tx(vf, kTileBytes);
         if (kt.kind == 0) {
           if (pair) {
-            tma_load_3d(sm.v, &maps.v, &sm.bar_vfull, 0, kt.j0 * 64, bh);
-            tma_load_3d(sm.v + kHalf, &maps.v, &sm.bar_vfull, 64, kt.j0 * 64, bh);
-            tma_load_3d(sm.v + 64 * 128, &maps.v, &sm.bar_vfull, 0, j1 * 64, bh);
-            tma_load_3d(sm.v + kHalf + 64 * 128, &maps.v, &sm.bar_vfull, 64, j1 * 64, bh);
+            tma_load_3d(vb, &maps.v, vf, 0, kt.j0 * 64, bh);
+            tma_load_3d(vb + kHalf, &maps.v, vf, 64, kt.j0 * 64, bh);
+            tma_load_3d(vb + 64 * 128, &maps.v, vf, 0, j1 * 64, bh);
+            tma_load_3d(vb + kHalf + 64 * 128, &maps.v, vf, 64, j1 * 64, bh);
           } else {
-            tma_load_3d(sm.v, &maps.v, &sm.bar_vfull, 0, kt.j0 * 128, bh);
-            tma_load_3d(sm.v + kHalf, &maps.v, &sm.bar_vfull, 64, kt.j0 * 128, bh);
+            tma_load_3d(vb, &maps.v, vf, 0, kt.j0 * 128, bh);
+            tma_load_3d(vb + kHalf, &maps.v, vf, 64, kt.j0 * 128, bh);
           }
         } else {
-          tma_load_3d(sm.v, &maps.vsum, &sm.bar_vfull, 0, kt.j0, bh);
-          tma_load_3d(sm.v + kHalf, &maps.vsum, &sm.bar_vfull, 64, kt.j0, bh);
+          tma_load_3d(vb, &maps.vsum, vf, 0, kt.j0, bh);
+          tma_load_3d(vb + kHalf, &maps.vsum, vf, 64, kt.j0, bh);
         }
         ++issued_v;
       }
       if (ok && need_corr) {
-        if ((ok = wait_or_abort(sm, &sm.bar_kempty, (T - 1) & 1, p))) {
-          mbar_expect_tx(&sm.bar_kfull, kTileBytes);
-          tma_load_3d(sm.k, &maps.hbar, &sm.bar_kfull, 0, 0, bh);
-          tma_load_3d(sm.k + kHalf, &maps.hbar, &sm.bar_kfull, 64, 0, bh);
+        const int ks = T % kKS;
+        if (T < kKS || (ok = wait_or_abort(sm, &sm.bar_kempty[ks], ((T / kKS) - 1) & 1, p))) {
+          mbar_expect_tx(&sm.bar_kfull[ks], kTileBytes);
+          tma_load_3d(sm.k[ks], &maps.hbar, &sm.bar_kfull[ks], 0, 0, bh);
+          tma_load_3d(sm.k[ks] + kHalf, &maps.hbar, &sm.bar_kfull[ks], 64, 0, bh);
           ++issued_k;
         }
       }
@@ -269,8 +288,10 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         // drain: every copy issued so far must land before this CTA's shared memory is released
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
-        while (issued_k > 0 && !mbar_try_wait(&sm.bar_kfull, (issued_k - 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
-        while (issued_v > 0 && !mbar_try_wait(&sm.bar_vfull, (issued_v - 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+        for (int i = max(0, issued_k - kKS); i < issued_k; ++i)
+          while (!mbar_try_wait(&sm.bar_kfull[i % kKS], (i / kKS) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+        for (int i = max(0, issued_v - kVS); i < issued_v; ++i)
+          while (!mbar_try_wait(&sm.bar_vfull[i % kVS], (i / kVS) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
       }
     }
   } else if (warp == 5) {
@@ -278,39 +299,43 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
-      const uint32_t q_addr = smem_u32(sm.q), k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+      const uint32_t q_addr = smem_u32(sm.q);
+      const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
       bool ok = wait_or_abort(sm, &sm.bar_q, 0, p);
       tc_fence_after();
       for (int t = 0; t < T && ok; ++t) {
-        if (!(ok = wait_or_abort(sm, &sm.bar_kfull, t & 1, p))) break;
+        const int ks = t % kKS, vs = t % kVS;
+        const uint32_t k_addr = smem_u32(sm.k[ks]), v_addr = smem_u32(sm.v[vs]);
+        if (!(ok = wait_or_abort(sm, &sm.bar_kfull[ks], (t / kKS) & 1, p))) break;
         tc_fence_after();
+        const uint64_t kd = smem_desc_sw128(k_addr, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tmem + kColS, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                 idesc_s, kk > 0);
+          const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;   // start-address field units
+          mma_ss(tmem + kColS, qd + off, kd + off, idesc_s, kk > 0);
         }
-        mma_commit(&sm.bar_kempty);
+        mma_commit(&sm.bar_kempty[ks]);
         mma_commit(&sm.bar_sfull);
         if (!(ok = wait_or_abort(sm, &sm.bar_pfull, t & 1, p))) break;
-        if (!(ok = wait_or_abort(sm, &sm.bar_vfull, t & 1, p))) break;
+        if (!(ok = wait_or_abort(sm, &sm.bar_vfull[vs], (t / kVS) & 1, p))) break;
         tc_fence_after();
+        const uint64_t vd = smem_desc_sw128(v_addr, kHalf, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(tmem + kColO, tmem + kColS + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024), idesc_pv,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&sm.bar_vempty);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + kColO, tmem + kColS + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_vempty[vs]);
         mma_commit(&sm.bar_odone);
       }
       if (ok && need_corr) {
-        if ((ok = wait_or_abort(sm, &sm.bar_kfull, T & 1, p))) {
+        const int ks = T % kKS;
+        const uint32_t k_addr = smem_u32(sm.k[ks]);
+        if ((ok = wait_or_abort(sm, &sm.bar_kfull[ks], (T / kKS) & 1, p))) {
           tc_fence_after();
+          const uint64_t kd = smem_desc_sw128(k_addr, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            mma_ss(tmem + kColS, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                   idesc_s, kk > 0);
+            const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + kColS, qd + off, kd + off, idesc_s, kk > 0);
           }
         }
       }
@@ -387,13 +412,13 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           for (int x = 0; x < 32; ++x) s[32 * g + x] = ((vm >> x) & 1u) ? s[32 * g + x] : -INFINITY;
         }
       }
-      float t0 = s[0], t1 = s[1], t2 = s[2], t3 = s[3];
+      float t0 = fmaxf(s[0], s[1]), t1 = fmaxf(s[2], s[3]), t2 = fmaxf(s[4], s[5]), t3 = fmaxf(s[6], s[7]);
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        t0 = fmaxf(t0, s[c]);
-        t1 = fmaxf(t1, s[c + 1]);
-        t2 = fmaxf(t2, s[c + 2]);
-        t3 = fmaxf(t3, s[c + 3]);
+      for (int c = 8; c < 128; c += 8) {
+        t0 = fmax3(t0, s[c], s[c + 1]);
+        t1 = fmax3(t1, s[c + 2], s[c + 3]);
+        t2 = fmax3(t2, s[c + 4], s[c + 5]);
+        t3 = fmax3(t3, s[c + 6], s[c + 7]);
       }
       const float m_new = fmaxf(m, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));   // raw logit units
       const bool grow = m_new > m;
@@ -412,19 +437,26 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       }
       // p = 2^(s*scale*log2e - m*scale*log2e); masked entries are -inf and give exactly 0
       const float mb = m == -INFINITY ? 0.f : m * p.scale_log2;
-      float ls = 0.f;
+      // exponents and row sums two at a time (f32x2 arithmetic)
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nmb2 = f2_pack(-mb, -mb);
+      uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          const float p0 = ex2(fmaf(s[32 * ch + x], p.scale_log2, -mb));
-          const float p1 = ex2(fmaf(s[32 * ch + x + 1], p.scale_log2, -mb));
-          ls += p0 + p1;
+          const int c = 32 * ch + x;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nmb2), x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          acc2 = f2_add(acc2, f2_pack(p0, p1));
           pk[x >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st16(trow + kColS + 16 * ch, pk);
       }
+      float ls0, ls1;
+      f2_unpack(acc2, ls0, ls1);
+      const float ls = ls0 + ls1;
       if (centroid) {
         // alpha of every unselected block enters D with weight cnt_j: `block` except the last one
         A += ls;
@@ -439,15 +471,14 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_odone, (t - 1) & 1, p));
         if (!ok) break;
         tc_fence_after();
+        float ov[128];               // the scores are dead here: one TMEM round trip for the whole row
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          float ov[32];
-          tmem_ld32(trow + kColO + 32 * ch, ov);
-          tmem_ld_wait();
+        for (int ch = 0; ch < 4; ++ch) tmem_ld32(trow + kColO + 32 * ch, ov + 32 * ch);
+        tmem_ld_wait();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) ov[x] *= f;
-          tmem_st32(trow + kColO + 32 * ch, ov);
-        }
+        for (int x = 0; x < 128; ++x) ov[x] *= f;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_st32(trow + kColO + 32 * ch, ov + 32 * ch);
       }
       tmem_st_wait();
       tc_fence_before();

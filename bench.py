@@ -35,6 +35,22 @@ def _peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def _profiled_traffic(workload: str):
+    """DRAM bytes of one attention launch from the committed ncu summary, if it was taken on the
+    attention kernel source as it is now (else None: the counters would be stale)."""
+    import glob
+    import hashlib
+    src = os.path.join(ROOT, "piecewise_approximate_attention_b200", "csrc", "attn_sm100.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"attn_sm100_{workload}-*.md"))):
+        text = open(path).read()
+        if f"source_sha256: {sha}" in text:
+            for line in text.splitlines():
+                if line.startswith("traffic_bytes_full_launch:"):
+                    return int(line.split(":")[1])
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples during the timed region."""
 
@@ -97,6 +113,25 @@ def effective_flops(sel, order_blocks_L: int, block: int, d: int, nb: int):
     return exact, centroid
 
 
+def aggregate(maxes, sums, device, world: int):
+    """Across ranks: element-wise max of `maxes` (times) and sum of `sums` (work).  With world == 1
+    the inputs come back unchanged; otherwise one all-reduce each, on whatever backend is up."""
+    if world <= 1:
+        return list(maxes), list(sums)
+    import torch
+    import torch.distributed as dist
+    a = torch.tensor(list(maxes), dtype=torch.float64, device=device)
+    b = torch.tensor(list(sums), dtype=torch.float64, device=device)
+    dist.all_reduce(a, op=dist.ReduceOp.MAX)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return a.tolist(), b.tolist()
+
+
+def rank_seed(w, rank: int) -> int:
+    """Each rank draws its own batch element: the workload seed offset by the rank."""
+    return w.seed + rank
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from piecewise_approximate_attention_b200 import _lib as C
@@ -107,7 +142,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     # each rank runs its own batch element: seed offset by rank
-    q, k, v = make_qkv(w, seed=w.seed + rank)
+    q, k, v = make_qkv(w, seed=rank_seed(w, rank))
     B, H, L, d = q.shape
     p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, dev)
     stream = torch.cuda.Stream(dev)
@@ -163,12 +198,7 @@ def run_ours(args, rank, world, local_rank):
     exact_fl, centroid_fl = effective_flops(p.sel, L, w.block, d, p.nb)
     corr_fl = 2.0 * L * d * d * B * H
     ms_step = total_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step, attn_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step, attn_ms_max = t.tolist()
-    else:
-        attn_ms_max = attn_ms
+    (ms_step, attn_ms_max), (exact_all,) = aggregate([ms_step, attn_ms], [exact_fl], dev, world)
 
     # library's own dense path (keep_k = nb) and exact-only mode, same GPU, outside the timed region
     dense = Pisa(B, H, L, d, w.block, p.nb, w.lam, w.dtype, 1.0, dev, pair=False)
@@ -218,17 +248,14 @@ def run_ours(args, rank, world, local_rank):
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
+    (e2e_ms,), _ = aggregate([e2e_ms], [], dev, world)
 
     peak, peak_sus, hbm, peak_kind = _peaks()
     attn_alg = exact_fl + centroid_fl + corr_fl
     achieved = attn_alg / (attn_ms * 1e-3) / 1e12
     result = {
         "metric": METRIC,
-        "value": round(world * exact_fl / (ms_step * 1e-3) / 1e12, 3),
+        "value": round(exact_all / (ms_step * 1e-3) / 1e12, 3),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -253,11 +280,11 @@ def run_ours(args, rank, world, local_rank):
         "attention_overhead_vs_exact_only": round(attn_ms / exact_only_ms - 1.0, 4),
         "effective_tflops_attention_only": round(exact_fl / (attn_ms * 1e-3) / 1e12, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": _profiled_traffic(w.name),
                      "kernel": "pisa_attention", "peak_kind": f"{peak_kind} bf16 dense burst",
                      "frac_of_sustained": round(achieved / peak_sus, 4),
                      "algorithmic_flops_per_launch": attn_alg},
-        "e2e": {"value": round(world * exact_fl / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(exact_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                 "d2h_bytes_per_step": o.numel() * o.element_size()},

@@ -41,7 +41,7 @@ constexpr int kThreads = 192;
 constexpr int kHalf = 128 * 64 * 2;        // one 128-row x 64-column bf16 half: 16 KB
 constexpr int kTileBytes = 2 * kHalf;      // 32 KB
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColO = 128;
+constexpr uint32_t kColS = 0, kColO = 128;   // S/P of the two 64-key halves at 0 and 64, O at 128
 constexpr int kWords = 128;                // selection bitmap words (nb <= 4096)
 #ifndef PISA_ATTN_KSTAGES
 #define PISA_ATTN_KSTAGES 1
@@ -57,7 +57,8 @@ struct alignas(1024) Smem {
   uint8_t q[kTileBytes];
   uint8_t k[kKS][kTileBytes];
   uint64_t bar_kfull[kKS], bar_kempty[kKS], bar_vfull[kVS], bar_vempty[kVS];
-  uint64_t bar_q, bar_sfull, bar_pfull, bar_odone, bar_final, bar_drain;
+  uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2];
+  uint64_t bar_q, bar_final, bar_drain;
   uint32_t tmem_base;
   int abort;
   int n_exact, n_cent, need_corr;
@@ -180,9 +181,11 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       mbar_init(&sm.bar_vfull[i], 1);
       mbar_init(&sm.bar_vempty[i], 1);
     }
-    mbar_init(&sm.bar_sfull, 1);
-    mbar_init(&sm.bar_pfull, 128);
-    mbar_init(&sm.bar_odone, 1);
+    for (int hh = 0; hh < 2; ++hh) {
+      mbar_init(&sm.bar_sfull[hh], 1);
+      mbar_init(&sm.bar_pfull[hh], 128);
+      mbar_init(&sm.bar_odone[hh], 1);
+    }
     mbar_init(&sm.bar_final, 1);
     mbar_init(&sm.bar_drain, 1);
     sm.abort = 0;
@@ -296,46 +299,66 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     }
   } else if (warp == 5) {
     // =============================== MMA issuer ===============================
+    // Each 128-key tile is two 64-key halves with their own S buffers, so the tensor core works on
+    // one half while the softmax warps work on the other:
+    //   S_a(0) S_b(0) | PV_a(0) S_a(1) PV_b(0) S_b(1) | PV_a(1) S_a(2) PV_b(1) S_b(2) | ...
+    // PV_h(t) reads P_h(t) from the S_h columns; S_h(t+1) overwrites them afterwards, in issue order.
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
-      const uint32_t q_addr = smem_u32(sm.q);
-      const uint64_t qd = smem_desc_sw128(q_addr, 16, 1024);
+      const uint32_t idesc_c = idesc_bf16_f32(128, 128, false, false);
+      const uint64_t qd = smem_desc_sw128(smem_u32(sm.q), 16, 1024);
       bool ok = wait_or_abort(sm, &sm.bar_q, 0, p);
       tc_fence_after();
-      for (int t = 0; t < T && ok; ++t) {
-        const int ks = t % kKS, vs = t % kVS;
-        const uint32_t k_addr = smem_u32(sm.k[ks]), v_addr = smem_u32(sm.v[vs]);
-        if (!(ok = wait_or_abort(sm, &sm.bar_kfull[ks], (t / kKS) & 1, p))) break;
-        tc_fence_after();
-        const uint64_t kd = smem_desc_sw128(k_addr, 16, 1024);
+      // S_h(t) = Q K_h(t)^T into columns 64h (keys 64h..64h+63 of tile t)
+      auto issue_s = [&](int t, int hh) -> bool {
+        const int ks = t % kKS;
+        if (hh == 0) {
+          if (!wait_or_abort(sm, &sm.bar_kfull[ks], (t / kKS) & 1, p)) return false;
+          tc_fence_after();
+        }
+        const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ks]) + 8192 * hh, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;   // start-address field units
-          mma_ss(tmem + kColS, qd + off, kd + off, idesc_s, kk > 0);
+          mma_ss(tmem + kColS + 64 * hh, qd + off, kd + off, idesc_s, kk > 0);
         }
-        mma_commit(&sm.bar_kempty[ks]);
-        mma_commit(&sm.bar_sfull);
-        if (!(ok = wait_or_abort(sm, &sm.bar_pfull, t & 1, p))) break;
-        if (!(ok = wait_or_abort(sm, &sm.bar_vfull[vs], (t / kVS) & 1, p))) break;
+        mma_commit(&sm.bar_sfull[hh]);
+        if (hh == 1) mma_commit(&sm.bar_kempty[ks]);
+        return true;
+      };
+      // O += P_h(t) V_h(t): P from TMEM columns 64h.., V rows 64h..64h+63 (MN-major)
+      auto issue_pv = [&](int t, int hh) -> bool {
+        const int vs = t % kVS;
+        if (!wait_or_abort(sm, &sm.bar_pfull[hh], t & 1, p)) return false;
+        if (hh == 0 && !wait_or_abort(sm, &sm.bar_vfull[vs], (t / kVS) & 1, p)) return false;
         tc_fence_after();
-        const uint64_t vd = smem_desc_sw128(v_addr, kHalf, 1024);
+        const uint64_t vd = smem_desc_sw128(smem_u32(sm.v[vs]) + 8192 * hh, kHalf, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + kColO, tmem + kColS + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.bar_vempty[vs]);
-        mma_commit(&sm.bar_odone);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + kColO, tmem + kColS + 64 * hh + kk * 8, vd + (uint64_t)(kk * 2048 >> 4), idesc_pv,
+                 (t > 0 || hh > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_odone[hh]);
+        if (hh == 1) mma_commit(&sm.bar_vempty[vs]);
+        return true;
+      };
+      if (ok && T > 0) ok = issue_s(0, 0) && issue_s(0, 1);
+      for (int t = 0; t < T && ok; ++t) {
+        ok = issue_pv(t, 0);
+        if (ok && t + 1 < T) ok = issue_s(t + 1, 0);
+        if (ok) ok = issue_pv(t, 1);
+        if (ok && t + 1 < T) ok = issue_s(t + 1, 1);
       }
       if (ok && need_corr) {
+        // Q (s Hbar^T) into columns 0..127, after every PV has read its P there
         const int ks = T % kKS;
-        const uint32_t k_addr = smem_u32(sm.k[ks]);
         if ((ok = wait_or_abort(sm, &sm.bar_kfull[ks], (T / kKS) & 1, p))) {
           tc_fence_after();
-          const uint64_t kd = smem_desc_sw128(k_addr, 16, 1024);
+          const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ks]), 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-            mma_ss(tmem + kColS, qd + off, kd + off, idesc_s, kk > 0);
+            mma_ss(tmem + kColS, qd + off, kd + off, idesc_c, kk > 0);
           }
         }
       }
@@ -347,8 +370,8 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     }
   } else {
     // =========================== softmax + epilogue ===========================
-    // Thread r owns tile row r (TMEM lane r).  Decisions that guard .sync.aligned TMEM accesses are
-    // made warp-uniform.
+    // Thread r owns tile row r (TMEM lane r) and walks the 64-key halves in MMA order.  Decisions
+    // that guard .sync.aligned TMEM accesses are made warp-uniform.
     const unsigned FULL = 0xffffffffu;
     const int r = threadIdx.x;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
@@ -360,61 +383,44 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     const float last_cnt = (float)block_count(p.nb - 1, p.L, p.block);
     float m = -INFINITY, l = 0.f, A = 0.f;
     UnionIter it;
+    KeyTile kt{0, 0, -1};
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_sfull, t & 1, p));
+    for (int u = 0; u < 2 * T; ++u) {
+      const int t = u >> 1, hh = u & 1;
+      ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_sfull[hh], t & 1, p));
       if (!ok) break;
       tc_fence_after();
-      const KeyTile kt = key_tile(t, n_exact, pair, it, sm.bitsA, sm.bitsB);
+      if (hh == 0) kt = key_tile(t, n_exact, pair, it, sm.bitsA, sm.bitsB);
       const bool centroid = kt.kind == 1;
-      float s[128];
-      tmem_ld32(trow + kColS + 0, s);
-      tmem_ld32(trow + kColS + 32, s + 32);
-      tmem_ld32(trow + kColS + 64, s + 64);
-      tmem_ld32(trow + kColS + 96, s + 96);
-      // column validity, 32 columns per word
-      uint32_t vmask[4];
+      float s[64];
+      tmem_ld32(trow + kColS + 64 * hh, s);
+      tmem_ld32(trow + kColS + 64 * hh + 32, s + 32);
+      // validity of this half's 64 columns, 32 per word
+      uint32_t vm0, vm1;
       if (!centroid) {
-        const int jh1 = pair ? kt.j1 : kt.j0;
-        const bool ok0 = kt.j0 >= 0 && bit_of(bits, kt.j0);
-        const bool ok1 = jh1 >= 0 && bit_of(bits, jh1);
-        const int c0 = ok0 ? block_count(kt.j0, p.L, p.block) : 0;
-        const int c1 = ok1 ? block_count(jh1, p.L, p.block) : 0;
-        if (pair) {
-          vmask[0] = c0 >= 32 ? FULL : ((1u << c0) - 1u);
-          vmask[1] = c0 >= 64 ? FULL : (c0 > 32 ? ((1u << (c0 - 32)) - 1u) : 0u);
-          vmask[2] = c1 >= 32 ? FULL : ((1u << c1) - 1u);
-          vmask[3] = c1 >= 64 ? FULL : (c1 > 32 ? ((1u << (c1 - 32)) - 1u) : 0u);
-        } else {
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int rem = c0 - 32 * g;
-            vmask[g] = rem >= 32 ? FULL : (rem > 0 ? ((1u << rem) - 1u) : 0u);
-          }
-        }
+        const int jh = pair ? (hh ? kt.j1 : kt.j0) : kt.j0;
+        const int cnt = (jh >= 0 && bit_of(bits, jh)) ? block_count(jh, p.L, p.block) : 0;
+        const int r0 = cnt - (pair ? 0 : 64 * hh), r1 = r0 - 32;   // valid columns left in each word
+        vm0 = r0 >= 32 ? FULL : (r0 > 0 ? ((1u << r0) - 1u) : 0u);
+        vm1 = r1 >= 32 ? FULL : (r1 > 0 ? ((1u << r1) - 1u) : 0u);
       } else {
-        const int w0 = kt.j0 >> 5;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int rem = p.nb - (kt.j0 + 32 * g);
-          const uint32_t inr = rem >= 32 ? FULL : (rem > 0 ? ((1u << rem) - 1u) : 0u);
-          vmask[g] = inr & ~(w0 + g < kWords ? bits[w0 + g] : 0u);
-        }
+        const int j0 = kt.j0 + 64 * hh, w0 = j0 >> 5;
+        const int r0 = p.nb - j0, r1 = r0 - 32;
+        vm0 = (r0 >= 32 ? FULL : (r0 > 0 ? ((1u << r0) - 1u) : 0u)) & ~(w0 < kWords ? bits[w0] : 0u);
+        vm1 = (r1 >= 32 ? FULL : (r1 > 0 ? ((1u << r1) - 1u) : 0u)) & ~(w0 + 1 < kWords ? bits[w0 + 1] : 0u);
       }
       tmem_ld_wait();
-      // masks touch only 32-column groups that are partly invalid (warp-uniform: a warp's 32 rows
-      // belong to one query block)
+      if (vm0 != FULL) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const uint32_t vm = vmask[g];
-        if (vm != FULL) {
+        for (int x = 0; x < 32; ++x) s[x] = ((vm0 >> x) & 1u) ? s[x] : -INFINITY;
+      }
+      if (vm1 != FULL) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) s[32 * g + x] = ((vm >> x) & 1u) ? s[32 * g + x] : -INFINITY;
-        }
+        for (int x = 0; x < 32; ++x) s[32 + x] = ((vm1 >> x) & 1u) ? s[32 + x] : -INFINITY;
       }
       float t0 = fmaxf(s[0], s[1]), t1 = fmaxf(s[2], s[3]), t2 = fmaxf(s[4], s[5]), t3 = fmaxf(s[6], s[7]);
 #pragma unroll
-      for (int c = 8; c < 128; c += 8) {
+      for (int c = 8; c < 64; c += 8) {
         t0 = fmax3(t0, s[c], s[c + 1]);
         t1 = fmax3(t1, s[c + 2], s[c + 3]);
         t2 = fmax3(t2, s[c + 4], s[c + 5]);
@@ -428,20 +434,20 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         A *= f;
         m = m_new;
       }
-      float slast = -INFINITY;     // raw logit of the last (short) key block, when this tile holds it
-      const int cl = p.nb - 1 - kt.j0;
-      const bool has_last = centroid && cl >= 0 && cl < 128 && last_cnt != (float)p.block;
+      float slast = -INFINITY;     // raw logit of the last (short) key block, when this half holds it
+      const int cl = p.nb - 1 - kt.j0 - 64 * hh;
+      const bool has_last = centroid && cl >= 0 && cl < 64 && last_cnt != (float)p.block;
       if (has_last) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) slast = c == cl ? s[c] : slast;
+        for (int c = 0; c < 64; ++c) slast = c == cl ? s[c] : slast;
       }
-      // p = 2^(s*scale*log2e - m*scale*log2e); masked entries are -inf and give exactly 0
+      // p = 2^(s*scale*log2e - m*scale*log2e) (masked entries are -inf and give exactly 0), two at a
+      // time with f32x2 arithmetic; P (bf16) goes over the first 32 columns of this half's S
       const float mb = m == -INFINITY ? 0.f : m * p.scale_log2;
-      // exponents and row sums two at a time (f32x2 arithmetic)
       const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nmb2 = f2_pack(-mb, -mb);
       uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
@@ -452,7 +458,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           acc2 = f2_add(acc2, f2_pack(p0, p1));
           pk[x >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(trow + kColS + 16 * ch, pk);
+        tmem_st16(trow + kColS + 64 * hh + 16 * ch, pk);
       }
       float ls0, ls1;
       f2_unpack(acc2, ls0, ls1);
@@ -465,24 +471,27 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       } else {
         l += ls;
       }
-      // O holds the PV products of earlier tiles (already complete: S(t) was committed after
-      // PV(t-1)); rescale it before PV(t) is released
-      if (__any_sync(FULL, grow) && t > 0) {
-        ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_odone, (t - 1) & 1, p));
+      // O holds the PV products of the earlier halves; rescale it before PV of this half is released.
+      // The previous half's PV was issued when its P was ready, long before this half's P was
+      // computed, so the wait below is normally already satisfied.
+      if (__any_sync(FULL, grow) && u > 0) {
+        const int ph = hh ^ 1, pt = hh ? t : t - 1;
+        ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_odone[ph], pt & 1, p));
         if (!ok) break;
         tc_fence_after();
-        float ov[128];               // the scores are dead here: one TMEM round trip for the whole row
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_ld32(trow + kColO + 32 * ch, ov + 32 * ch);
-        tmem_ld_wait();
+        for (int ch = 0; ch < 4; ++ch) {
+          float ov[32];
+          tmem_ld32(trow + kColO + 32 * ch, ov);
+          tmem_ld_wait();
 #pragma unroll
-        for (int x = 0; x < 128; ++x) ov[x] *= f;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_st32(trow + kColO + 32 * ch, ov + 32 * ch);
+          for (int x = 0; x < 32; ++x) ov[x] *= f;
+          tmem_st32(trow + kColO + 32 * ch, ov);
+        }
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sm.bar_pfull);
+      mbar_arrive(&sm.bar_pfull[hh]);
     }
     if (ok) ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_final, 0, p));
     if (ok) {

@@ -18,7 +18,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kRows = 4;          // query blocks per CTA
 
 __device__ __forceinline__ float warp_max(float x) {
   for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
@@ -90,14 +89,23 @@ __device__ void warp_topk(const uint32_t* u, int nb, int keep_k, uint32_t* hist,
   }
 }
 
-template <int D>
+// Scores of kRows query blocks against all nb centroids: k̄ is streamed through shared memory in
+// tiles of kTileJ = 4 * kThreads / kRows rows (coalesced float4 loads, rows padded by 4 floats so
+// the float4 reads of 32 different rows are conflict-free); each thread accumulates 4 query blocks
+// x 1 centroid.
+template <int kRows>
+constexpr int tile_j() { return 4 * kThreads / kRows; }
+
+template <int D, int kRows>
 __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
                                                          const float* __restrict__ M, int L, int block, int nb,
                                                          float scale, int keep_k, float lam,
                                                          int32_t* __restrict__ sel, float* __restrict__ scores) {
-  extern __shared__ float smem[];
+  constexpr int kTileJ = tile_j<kRows>();
+  extern __shared__ __align__(16) float smem[];
   float* qs = smem;                                        // [kRows][D]
-  float* r = qs + kRows * D;                               // [kRows][nb]
+  float* ks = qs + kRows * D;                              // [kTileJ][D + 4]
+  float* r = ks + kTileJ * (D + 4);                        // [kRows][nb]
   uint32_t* hist = reinterpret_cast<uint32_t*>(r + kRows * nb);   // [kWarps][256]
   float* red = reinterpret_cast<float*>(hist + kWarps * 256);     // [kWarps]
   const int bh = blockIdx.y, i0 = blockIdx.x * kRows;
@@ -114,28 +122,38 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
   for (int j = threadIdx.x; j < nb; j += kThreads) msum += Mh[j];
   msum = warp_sum(msum);
   if (lane == 0) red[warp] = msum;
+
+  const int jj = threadIdx.x % kTileJ, g = threadIdx.x / kTileJ;   // centroid column, query group
+  const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nb * D);
+  for (int j0 = 0; j0 < nb; j0 += kTileJ) {
+    const int nj = min(kTileJ, nb - j0);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < kTileJ * (D / 4); idx += kThreads) {
+      const int jr = idx / (D / 4), a4 = idx % (D / 4);
+      const float4 v = jr < nj ? kb4[(size_t)(j0 + jr) * (D / 4) + a4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(ks + jr * (D + 4) + 4 * a4) = v;
+    }
+    __syncthreads();
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* kr = ks + jj * (D + 4);
+#pragma unroll 8
+    for (int a = 0; a < D; a += 4) {
+      const float4 kv = *reinterpret_cast<const float4*>(kr + a);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + (4 * g + x) * D + a);
+        acc[x] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, acc[x]))));
+      }
+    }
+    if (jj < nj) {
+#pragma unroll
+      for (int x = 0; x < 4; ++x) r[(4 * g + x) * nb + j0 + jj] = acc[x];
+    }
+  }
   __syncthreads();
   msum = 0.f;
   for (int w = 0; w < kWarps; ++w) msum += red[w];
   const float minv = msum > 0.f ? lam / msum : 0.f;
-
-  const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nb * D);
-  for (int j = threadIdx.x; j < nb; j += kThreads) {
-    float acc[kRows];
-#pragma unroll
-    for (int ri = 0; ri < kRows; ++ri) acc[ri] = 0.f;
-    for (int a4 = 0; a4 < D / 4; ++a4) {
-      const float4 kv = kb4[(size_t)j * (D / 4) + a4];
-#pragma unroll
-      for (int ri = 0; ri < kRows; ++ri) {
-        const float* qq = qs + ri * D + 4 * a4;
-        acc[ri] = fmaf(qq[0], kv.x, fmaf(qq[1], kv.y, fmaf(qq[2], kv.z, fmaf(qq[3], kv.w, acc[ri]))));
-      }
-    }
-#pragma unroll
-    for (int ri = 0; ri < kRows; ++ri) r[ri * nb + j] = acc[ri];
-  }
-  __syncthreads();
 
   const float last_cnt = (float)(L - (nb - 1) * block);
   for (int ri = warp; ri < rows; ri += kWarps) {
@@ -249,24 +267,32 @@ __global__ void identity_order(int nb, int32_t* __restrict__ order) {
     order[(size_t)bh * nb + i] = i;
 }
 
+template <int D, int kRows>
+cudaError_t launch_route_kernel(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
+                                float* scores, cudaStream_t stream) {
+  const size_t smem = ((size_t)kRows * D + (size_t)tile_j<kRows>() * (D + 4) + (size_t)kRows * g.nb) * sizeof(float) +
+                      kWarps * 256 * sizeof(uint32_t) + kWarps * sizeof(float);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(route_kernel<D, kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+    return e;
+  route_kernel<D, kRows><<<dim3((g.nb + kRows - 1) / kRows, g.BH()), kThreads, smem, stream>>>(
+      st.qbar, st.kbar, st.M, g.L, g.block, g.nb, g.scale, keep_k, lam, sel, scores);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream) {
-  const size_t smem = ((size_t)kRows * g.d + (size_t)kRows * g.nb) * sizeof(float) + kWarps * 256 * sizeof(uint32_t) +
-                      kWarps * sizeof(float);
-  dim3 grid((g.nb + kRows - 1) / kRows, g.BH());
   cudaError_t e;
-  if (g.d == 64) {
-    if ((e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
-    route_kernel<64><<<grid, kThreads, smem, stream>>>(st.qbar, st.kbar, st.M, g.L, g.block, g.nb, g.scale, keep_k,
-                                                        lam, sel, scores);
-  } else {
-    if ((e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
-    route_kernel<128><<<grid, kThreads, smem, stream>>>(st.qbar, st.kbar, st.M, g.L, g.block, g.nb, g.scale, keep_k,
-                                                         lam, sel, scores);
-  }
-  if ((e = cudaGetLastError())) return e;
+  // 16 query blocks per CTA while their score rows fit comfortably in shared memory, else 8
+  if (g.d == 64)
+    e = g.nb <= 2048 ? launch_route_kernel<64, 16>(g, st, keep_k, lam, sel, scores, stream)
+                     : launch_route_kernel<64, 8>(g, st, keep_k, lam, sel, scores, stream);
+  else
+    e = g.nb <= 2048 ? launch_route_kernel<128, 16>(g, st, keep_k, lam, sel, scores, stream)
+                     : launch_route_kernel<128, 8>(g, st, keep_k, lam, sel, scores, stream);
+  if (e != cudaSuccess) return e;
   if (order) {
     if (g.block == 64 && keep_k > 0 && g.nb > 2) {
       const int nwords = (g.nb + 31) / 32;

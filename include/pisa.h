@@ -71,8 +71,11 @@ typedef struct {
 } pisa_shape;
 
 /* Per-head block statistics written by pisa_precompute.  nb = pisa_num_blocks(L, block).
- * All fp32 arrays are dense row-major.  The *_op arrays are tensor-core operand copies and are
- * used (and must be non-null) only when dtype == PISA_BF16. */
+ * All fp32 arrays are dense row-major.  The *_op arrays and vscale are tensor-core operand copies
+ * and are used (and must be non-null) only when dtype == PISA_BF16: the softmax weights and the
+ * values meet in an fp16 product (11 significant bits for the weights instead of bf16's 8), so the
+ * values get an fp16 copy scaled by a per-head power of two that keeps every sum of a block in
+ * range. */
 typedef struct {
   float* qbar;     /* [B,H,nb,d]  mean of q over query block i                                */
   float* kbar;     /* [B,H,nb,d]  centroid of key block j                                      */
@@ -81,8 +84,10 @@ typedef struct {
   float* M;        /* [B,H,nb]    ||H_j - Hbar||_F                                             */
   float* H;        /* nullable [B,H,nb,d,d]: per-block H_j, written only when non-null         */
   void*  kbar_op;  /* bf16 [B,H,nb,d]  kbar rounded to bf16                                    */
-  void*  vsum_op;  /* bf16 [B,H,nb,d]  vsum rounded to bf16                                    */
+  void*  vsum_op;  /* fp16 [B,H,nb,d]  vsum / vscale, rounded to fp16                          */
   void*  hbar_op;  /* bf16 [B,H,d,d]   softmax_scale * Hbar^T, i.e. hbar_op[c][a]              */
+  void*  v_op;     /* fp16 [B,H,L,d]   v / vscale (exact for every bf16 value in fp16 range)   */
+  float* vscale;   /* [B,H]            power of two >= max|v| / 256 (1 when max|v| <= 256)     */
 } pisa_stats;
 
 /* ABI revision of this header. */
@@ -92,7 +97,7 @@ PISA_API int32_t pisa_abi_version(void);
 PISA_API int32_t pisa_num_blocks(int32_t seq_len, int32_t block);
 
 /* Bytes of one contiguous buffer that pisa_stats_carve can split into every pisa_stats array
- * (H included when with_H != 0).  0 if the shape is invalid. */
+ * (H included when with_H != 0; the operand copies only for PISA_BF16).  0 if the shape is invalid. */
 PISA_API size_t pisa_stats_bytes(const pisa_shape* shape, int32_t with_H);
 
 /* Host-only pointer arithmetic: fills *out with 256-byte-aligned sub-ranges of [base, base+bytes).

@@ -31,7 +31,7 @@ class PisaShape(ctypes.Structure):
 
 class PisaStats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("qbar", "kbar", "vsum", "hbar", "M", "H", "kbar_op", "vsum_op", "hbar_op")]
+                ("qbar", "kbar", "vsum", "hbar", "M", "H", "kbar_op", "vsum_op", "hbar_op", "v_op", "vscale")]
 
 
 class PisaError(RuntimeError):
@@ -134,6 +134,8 @@ class Stats:
     kbar_op: object
     vsum_op: object
     hbar_op: object
+    v_op: object
+    vscale: object
 
 
 def alloc_stats(shape: PisaShape, device, with_H: bool = False) -> Stats:
@@ -159,11 +161,12 @@ def alloc_stats(shape: PisaShape, device, with_H: bool = False) -> Stats:
         esz = torch.empty((), dtype=dtype).element_size()
         return buf[off:off + numel * esz].view(dtype).view(*dims)
 
-    f32, bf = torch.float32, torch.bfloat16
+    f32, bf, f16 = torch.float32, torch.bfloat16, torch.float16
     return Stats(buf, st, view(st.qbar, f32, (B, H, nb, d)), view(st.kbar, f32, (B, H, nb, d)),
                  view(st.vsum, f32, (B, H, nb, d)), view(st.hbar, f32, (B, H, d, d)), view(st.M, f32, (B, H, nb)),
                  view(st.H, f32, (B, H, nb, d, d)), view(st.kbar_op, bf, (B, H, nb, d)),
-                 view(st.vsum_op, bf, (B, H, nb, d)), view(st.hbar_op, bf, (B, H, d, d)))
+                 view(st.vsum_op, f16, (B, H, nb, d)), view(st.hbar_op, bf, (B, H, d, d)),
+                 view(st.v_op, f16, (B, H, shape.seq_len, d)), view(st.vscale, f32, (B, H)))
 
 
 def alloc_workspace(shape: PisaShape, device):

@@ -43,7 +43,7 @@ pisa_status check_stats(const Dims& g, const pisa_stats* st, bool need_ops) {
     if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
   if (st->H && !aligned16(st->H)) return PISA_ERR_INVALID_ARG;
   if (need_ops && g.dtype == PISA_BF16) {
-    const void* ops[] = {st->kbar_op, st->vsum_op, st->hbar_op};
+    const void* ops[] = {st->kbar_op, st->vsum_op, st->hbar_op, st->v_op, st->vscale};
     for (const void* p : ops)
       if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
   }
@@ -54,18 +54,23 @@ pisa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PISA_OK : PIS
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+constexpr int kStatsArrays = 11;
+
 // Sizes of the stats arrays in carve order.
-void stats_sizes(const Dims& g, int with_H, size_t out[9]) {
+void stats_sizes(const Dims& g, int with_H, size_t out[kStatsArrays]) {
   const size_t bh = (size_t)g.BH(), nb = (size_t)g.nb, d = (size_t)g.d;
+  const bool ops = g.dtype == PISA_BF16;
   out[0] = bh * nb * d * 4;            // qbar
   out[1] = bh * nb * d * 4;            // kbar
   out[2] = bh * nb * d * 4;            // vsum
   out[3] = bh * d * d * 4;             // hbar
   out[4] = bh * nb * 4;                // M
   out[5] = with_H ? bh * nb * d * d * 4 : 0;  // H
-  out[6] = bh * nb * d * 2;            // kbar_op
-  out[7] = bh * nb * d * 2;            // vsum_op
-  out[8] = bh * d * d * 2;             // hbar_op
+  out[6] = ops ? bh * nb * d * 2 : 0;  // kbar_op
+  out[7] = ops ? bh * nb * d * 2 : 0;  // vsum_op
+  out[8] = ops ? bh * d * d * 2 : 0;   // hbar_op
+  out[9] = ops ? bh * (size_t)g.L * d * 2 : 0;   // v_op
+  out[10] = ops ? bh * 4 : 0;          // vscale
 }
 
 }  // namespace
@@ -75,7 +80,7 @@ using namespace pisa;
 
 extern "C" {
 
-int32_t pisa_abi_version(void) { return 1; }
+int32_t pisa_abi_version(void) { return 2; }
 
 int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
   if (seq_len < 1 || block < 1) return -1;
@@ -85,7 +90,7 @@ int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
 size_t pisa_stats_bytes(const pisa_shape* shape, int32_t with_H) {
   Dims g;
   if (check_shape(shape, &g) != PISA_OK) return 0;
-  size_t sz[9];
+  size_t sz[kStatsArrays];
   stats_sizes(g, with_H, sz);
   size_t tot = 0;
   for (size_t s : sz) tot += round_up(s, 256);
@@ -98,11 +103,11 @@ pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, 
   if (s != PISA_OK) return s;
   if (!base || !out || (reinterpret_cast<uintptr_t>(base) & 255u)) return PISA_ERR_INVALID_ARG;
   if (bytes < pisa_stats_bytes(shape, with_H)) return PISA_ERR_INVALID_ARG;
-  size_t sz[9];
+  size_t sz[kStatsArrays];
   stats_sizes(g, with_H, sz);
   char* p = static_cast<char*>(base);
-  void* ptr[9];
-  for (int i = 0; i < 9; ++i) {
+  void* ptr[kStatsArrays];
+  for (int i = 0; i < kStatsArrays; ++i) {
     ptr[i] = sz[i] ? p : nullptr;
     p += round_up(sz[i], 256);
   }
@@ -116,6 +121,8 @@ pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, 
   st.kbar_op = ptr[6];
   st.vsum_op = ptr[7];
   st.hbar_op = ptr[8];
+  st.v_op = ptr[9];
+  st.vscale = static_cast<float*>(ptr[10]);
   *out = st;
   return PISA_OK;
 }
@@ -123,7 +130,7 @@ pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, 
 size_t pisa_workspace_bytes(const pisa_shape* shape) {
   Dims g;
   if (check_shape(shape, &g) != PISA_OK) return 0;
-  return kStatusBytes + round_up(partials_bytes(g), 256);
+  return kStatusBytes + round_up(partials_bytes(g), 256) + round_up(vmax_bytes(g), 256);
 }
 
 pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
@@ -174,12 +181,13 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
     AttnMaps maps;
     const uint64_t bh = (uint64_t)g.BH();
     if (!encode_bf16_3d(&maps.q, q, g.d, g.L, bh, g.block) || !encode_bf16_3d(&maps.k, k, g.d, g.L, bh, g.block) ||
-        !encode_bf16_3d(&maps.v, v, g.d, g.L, bh, g.block) ||
+        !encode_16bit_3d(&maps.v, stats->v_op, g.d, g.L, bh, g.block, true) ||
         !encode_bf16_3d(&maps.kbar, stats->kbar_op, g.d, g.nb, bh, 128) ||
-        !encode_bf16_3d(&maps.vsum, stats->vsum_op, g.d, g.nb, bh, 128) ||
+        !encode_16bit_3d(&maps.vsum, stats->vsum_op, g.d, g.nb, bh, 128, true) ||
         !encode_bf16_3d(&maps.hbar, stats->hbar_op, g.d, g.d, bh, 128))
       return PISA_ERR_CUDA;
-    return cuda_status(launch_attention_sm100(g, maps, sel, order, keep_k, mode, o, status, kWaitLimitNs, cs));
+    return cuda_status(
+        launch_attention_sm100(g, maps, sel, order, keep_k, mode, stats->vscale, o, status, kWaitLimitNs, cs));
   }
   return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status, cs));
 }

@@ -18,10 +18,11 @@
 //     masked).  Both kinds run through the same tcgen05 MMAs: S = Q K^T into TMEM (fp32), softmax in
 //     registers (one thread per row), P (bf16) written back over S in TMEM, O += P V with P read from
 //     TMEM and V from shared memory (MN-major).
-//   * The running max is updated whenever a tile raises it, with O rescaled in TMEM.  The largest
-//     weight of a row is then exactly 1.0 in bf16, which keeps rows dominated by one key accurate
-//     (a max that lags by up to 2^8 measured ~10x larger errors on such rows).  The tcgen05.commit
-//     that signals S(t) also covers PV(t-1), so a rescale never waits on the tensor core.
+//   * P enters the PV product in fp16 (11 significant bits) against an fp16 copy of the values
+//     (v / vscale, a per-head power of two, written by the pre-computation).  That precision lets
+//     the running max lag the true row max by up to 2^8 (weights up to 256), so O is rescaled in
+//     TMEM only when a row max jumps by more than that; with bf16 weights the lag measured ~10x
+//     larger errors on rows dominated by one key.  The epilogue multiplies O back by vscale.
 //   * The correction is one more MMA, Q (s Hbar^T), into the S columns after the last PV; the
 //     epilogue computes o = (O + A * (Q s Hbar)) / l with A = sum of alpha over U_i.
 // Warp roles: warps 0-3 softmax + epilogue (TMEM lanes 0-127), warp 4 TMA producer, warp 5 MMA
@@ -43,6 +44,7 @@ constexpr int kTileBytes = 2 * kHalf;      // 32 KB
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColO = 128;   // S/P of the two 64-key halves at 0 and 64, O at 128
 constexpr int kWords = 128;                // selection bitmap words (nb <= 4096)
+constexpr float kLazyLog2 = 8.f;           // the running max may lag by 2^8 (fp16 weights up to 256)
 #ifndef PISA_ATTN_KSTAGES
 #define PISA_ATTN_KSTAGES 1
 #endif
@@ -69,6 +71,8 @@ struct alignas(1024) Smem {
 struct Params {
   int L, nb, block, keep_k, mode, dense;
   float scale_log2;
+  float lazy;                // rescale O only when the row max grows by more than this (logit units)
+  const float* vscale;       // [B*H] value scale of the fp16 value operands
   const int32_t* sel;
   const int32_t* order;
   __nv_bfloat16* o;
@@ -305,7 +309,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     // PV_h(t) reads P_h(t) from the S_h columns; S_h(t+1) overwrites them afterwards, in issue order.
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      const uint32_t idesc_pv = idesc_f16_f32(128, 128, false, true);
       const uint32_t idesc_c = idesc_bf16_f32(128, 128, false, false);
       const uint64_t qd = smem_desc_sw128(smem_u32(sm.q), 16, 1024);
       bool ok = wait_or_abort(sm, &sm.bar_q, 0, p);
@@ -427,7 +431,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         t3 = fmax3(t3, s[c + 6], s[c + 7]);
       }
       const float m_new = fmaxf(m, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));   // raw logit units
-      const bool grow = m_new > m;
+      const bool grow = m_new > m + p.lazy;
       const float f = grow ? ex2((m - m_new) * p.scale_log2) : 1.f;   // 0 when m = -inf
       if (grow) {
         l *= f;
@@ -456,7 +460,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nmb2), x0, x1);
           const float p0 = ex2(x0), p1 = ex2(x1);
           acc2 = f2_add(acc2, f2_pack(p0, p1));
-          pk[x >> 1] = pack_bf16x2(p0, p1);
+          pk[x >> 1] = pack_f16x2(p0, p1);
         }
         tmem_st16(trow + kColS + 64 * hh + 16 * ch, pk);
       }
@@ -496,7 +500,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     if (ok) ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_final, 0, p));
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / l, vsc = p.vscale[bh];
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.L + (size_t)myq * p.block + rloc) * D;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
@@ -507,7 +511,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          float a = ov[x], b = ov[x + 1];
+          float a = ov[x] * vsc, b = ov[x + 1] * vsc;
           if (need_corr) {
             a = fmaf(A, cv[x], a);
             b = fmaf(A, cv[x + 1], b);
@@ -534,8 +538,8 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
 size_t attention_sm100_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
-                                   int keep_k, int mode, void* o, int* status, unsigned long long wait_ns,
-                                   cudaStream_t stream) {
+                                   int keep_k, int mode, const float* vscale, void* o, int* status,
+                                   unsigned long long wait_ns, cudaStream_t stream) {
   Params p;
   p.L = g.L;
   p.nb = g.nb;
@@ -544,6 +548,8 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
   p.mode = mode;
   p.dense = keep_k == g.nb;
   p.scale_log2 = g.scale * 1.4426950408889634f;
+  p.lazy = kLazyLog2 / p.scale_log2;
+  p.vscale = vscale;
   p.sel = sel;
   p.order = order;
   p.o = static_cast<__nv_bfloat16*>(o);

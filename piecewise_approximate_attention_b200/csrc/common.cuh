@@ -26,6 +26,9 @@ inline int num_parts(const Dims& g) { return (g.nb + kBlocksPerPart - 1) / kBloc
 inline size_t partials_bytes(const Dims& g) {
   return (size_t)g.BH() * num_parts(g) * g.d * g.d * sizeof(float);
 }
+// after the partials: per (head, group of blocks) max |v|, which sets the head's value scale
+inline size_t vmax_bytes(const Dims& g) { return (size_t)g.BH() * num_parts(g) * sizeof(float); }
+inline size_t vmax_offset(const Dims& g) { return kStatusBytes + ((partials_bytes(g) + 255) / 256) * 256; }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -55,6 +58,9 @@ struct AttnMaps {
 // 128-byte swizzling; false if the driver entry point is unavailable or rejects the arguments.
 bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
                     uint32_t box_rows);
+// Same for a bf16 (fp16 == false) or fp16 (fp16 == true) tensor.
+bool encode_16bit_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                     uint32_t box_rows, bool fp16);
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits: 2 s
 
@@ -63,13 +69,13 @@ cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, 
                                    const pisa_stats& st, void* ws, cudaStream_t stream);
 cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v,
                                     const pisa_stats& st, void* ws, cudaStream_t stream);
-cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const pisa_stats& st,
-                               cudaStream_t stream);
+cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const float* vmax,
+                               const pisa_stats& st, cudaStream_t stream);
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream);
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
-                                   int keep_k, int mode, void* o, int* status, unsigned long long wait_ns,
-                                   cudaStream_t stream);
+                                   int keep_k, int mode, const float* vscale, void* o, int* status,
+                                   unsigned long long wait_ns, cudaStream_t stream);
 cudaError_t launch_attention_simt(const Dims& g, const void* q, const void* k, const void* v,
                                   const pisa_stats& st, const int32_t* sel, int keep_k, int mode,
                                   void* o, int* status, cudaStream_t stream);

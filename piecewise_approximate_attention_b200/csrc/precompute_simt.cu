@@ -88,8 +88,6 @@ __global__ void __launch_bounds__(kThreads) stats_partial(const T* __restrict__ 
       st.kbar[so + c] = kb[c];
       st.vsum[so + c] = vb[c];
       st.qbar[so + c] = qb[c];
-      if (st.kbar_op) reinterpret_cast<__nv_bfloat16*>(st.kbar_op)[so + c] = __float2bfloat16_rn(kb[c]);
-      if (st.vsum_op) reinterpret_cast<__nv_bfloat16*>(st.vsum_op)[so + c] = __float2bfloat16_rn(vb[c]);
     }
     accumulate_H<D>(Ks, Vs, block_count(j, L, block), acc);
     __syncthreads();
@@ -101,11 +99,22 @@ __global__ void __launch_bounds__(kThreads) stats_partial(const T* __restrict__ 
   for (int r = 0; r < R; ++r) out[(a0 + r * kStep) * D + c] = acc[r];
 }
 
+// Per head: Hbar = (sum of the group partials of H_j, in order) / nb, its bf16 operand copy, and
+// (when vmax is given) the value scale: the smallest power of two >= max|v| / 256, so that
+// v / vscale and every block sum of it (at most 128 terms) fit comfortably in fp16.
 template <int D>
 __global__ void __launch_bounds__(kThreads) hbar_reduce(const float* __restrict__ partials, int nparts, int nb,
                                                         float scale, float* __restrict__ hbar,
-                                                        __nv_bfloat16* __restrict__ hbar_op) {
+                                                        __nv_bfloat16* __restrict__ hbar_op,
+                                                        const float* __restrict__ vmax, float* __restrict__ vscale) {
   const int e = blockIdx.x * kThreads + threadIdx.x, bh = blockIdx.y;
+  if (vmax && vscale && blockIdx.x == 0 && threadIdx.x == 0) {
+    float mx = 0.f;
+    for (int i = 0; i < nparts; ++i) mx = fmaxf(mx, vmax[(size_t)bh * nparts + i]);
+    float sc = 1.f;
+    while (mx > 256.f * sc && sc < 0x1p100f) sc *= 2.f;
+    vscale[bh] = sc;
+  }
   if (e >= D * D) return;
   const float* p = partials + (size_t)bh * nparts * D * D + e;
   float s = 0.f;
@@ -171,7 +180,7 @@ cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, cons
   stats_partial<T, D><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g.L, g.block, g.nb, st, partials);
   hbar_reduce<D><<<dim3((D * D + kThreads - 1) / kThreads, g.BH()), kThreads, 0, stream>>>(
-      partials, nparts, g.nb, g.scale, st.hbar, static_cast<__nv_bfloat16*>(st.hbar_op));
+      partials, nparts, g.nb, g.scale, st.hbar, static_cast<__nv_bfloat16*>(st.hbar_op), nullptr, nullptr);
   cov_norm<T, D><<<dim3(g.nb, g.BH()), kThreads, smem_c, stream>>>(
       static_cast<const T*>(k), static_cast<const T*>(v), g.L, g.block, g.nb, st);
   return cudaGetLastError();
@@ -179,15 +188,15 @@ cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, cons
 
 }  // namespace
 
-cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const pisa_stats& st,
-                               cudaStream_t stream) {
+cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const float* vmax,
+                               const pisa_stats& st, cudaStream_t stream) {
   dim3 grid((g.d * g.d + kThreads - 1) / kThreads, g.BH());
   if (g.d == 64)
     hbar_reduce<64><<<grid, kThreads, 0, stream>>>(partials, nparts, g.nb, g.scale, st.hbar,
-                                                   static_cast<__nv_bfloat16*>(st.hbar_op));
+                                                   static_cast<__nv_bfloat16*>(st.hbar_op), vmax, st.vscale);
   else
     hbar_reduce<128><<<grid, kThreads, 0, stream>>>(partials, nparts, g.nb, g.scale, st.hbar,
-                                                    static_cast<__nv_bfloat16*>(st.hbar_op));
+                                                    static_cast<__nv_bfloat16*>(st.hbar_op), vmax, st.vscale);
   return cudaGetLastError();
 }
 

@@ -11,10 +11,14 @@
 // accumulates sum_n k_n v_n^T over the whole group in TMEM with tcgen05 (both operands MN-major,
 // fp32 accumulate).  Its epilogue subtracts sum_j kbar_j vsum_j^T, giving the group's partial
 // sum_j H_j.  The fixed-order reduction of the partials (hbar_reduce) gives Hbar.
-// Pass B (one CTA per head and group of key blocks): re-streams K, V, recomputes each H_j with one
-// MMA chain per block into double-buffered TMEM and reduces ||H_j - kbar_j vsum_j^T - Hbar||^2 in
-// the epilogue.  Re-reading K, V (2 L d bf16) costs less HBM traffic than storing and re-reading
+// Pass A also reduces max |v| per group; hbar_reduce turns it into the head's value scale (a power
+// of two).  Pass B (one CTA per head and group of key blocks): re-streams K, V, recomputes each H_j
+// with one MMA chain per block into double-buffered TMEM and reduces ||H_j - kbar_j vsum_j^T -
+// Hbar||^2 in the epilogue, and writes the attention's fp16 value operands v / vscale and
+// vsum / vscale from the tiles it streams.  Re-reading K, V (2 L d bf16) costs less HBM traffic than storing and re-reading
 // H_j (nb d^2 fp32).
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -54,8 +58,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, int* ab
 }
 
 // Sums of 8 consecutive columns (chunk cc of 16) over the rows r in [r0, r1) with r = rg (mod 8), read
-// from a 128B-swizzled [128 x 128] bf16 tile.  r0 is a multiple of 8.
-__device__ __forceinline__ void colsum8(const uint8_t* tile, int cc, int rg, int r0, int r1, float acc[8]) {
+// from a 128B-swizzled [128 x 128] bf16 tile.  r0 is a multiple of 8.  amax (if given) tracks max |x|.
+__device__ __forceinline__ void colsum8(const uint8_t* tile, int cc, int rg, int r0, int r1, float acc[8],
+                                        float* amax = nullptr) {
   const uint8_t* base = tile + (cc >> 3) * kHalf + (((cc & 7) ^ rg) << 4);
 #pragma unroll 4
   for (int r = r0 + rg; r < r1; r += 8) {
@@ -68,6 +73,16 @@ __device__ __forceinline__ void colsum8(const uint8_t* tile, int cc, int rg, int
     acc[5] += __uint_as_float(u.z & 0xffff0000u);
     acc[6] += __uint_as_float(u.w << 16);
     acc[7] += __uint_as_float(u.w & 0xffff0000u);
+    if (amax) {
+      // |x| of two packed bf16 at once: clear both sign bits; the larger magnitude sets the max
+      const uint32_t a0 = u.x & 0x7fff7fffu, a1 = u.y & 0x7fff7fffu, a2 = u.z & 0x7fff7fffu, a3 = u.w & 0x7fff7fffu;
+      float m = *amax;
+      m = fmaxf(m, fmaxf(__uint_as_float(a0 << 16), __uint_as_float(a0 & 0xffff0000u)));
+      m = fmaxf(m, fmaxf(__uint_as_float(a1 << 16), __uint_as_float(a1 & 0xffff0000u)));
+      m = fmaxf(m, fmaxf(__uint_as_float(a2 << 16), __uint_as_float(a2 & 0xffff0000u)));
+      m = fmaxf(m, fmaxf(__uint_as_float(a3 << 16), __uint_as_float(a3 & 0xffff0000u)));
+      *amax = m;
+    }
   }
 }
 
@@ -79,6 +94,7 @@ struct PreParams {
   int L, nb, block;
   pisa_stats st;
   float* partials;
+  float* vmax;               // [BH][nparts] max |v| per group (pass A)
   int* status;
   unsigned long long wait_ns;
 };
@@ -174,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
     for (int c = 0; c < D; ++c) corr[c] = 0.f;
     bool ok = true;
     int nblk = 0;
+    float vabs = 0.f;
     for (int t = 0; t < ntile; ++t) {
       const int s = t & 1;
       ok = !epi_any_failed(!wait_bar(&sm.full[s], (t >> 1) & 1, &sm.abort, p.status, p.wait_ns));
@@ -186,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
         float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0}, av[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         colsum8(sm.q[s], cc, rg, r0, r0 + cnt, aq);
         colsum8(sm.k[s], cc, rg, r0, r0 + cnt, ak);
-        colsum8(sm.v[s], cc, rg, r0, r0 + cnt, av);
+        colsum8(sm.v[s], cc, rg, r0, r0 + cnt, av, &vabs);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
           sm.red[0][rg][cc * 8 + x] = aq[x];
@@ -208,7 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
         p.st.kbar[so] = sk * inv;
         p.st.vsum[so] = sv;
         reinterpret_cast<__nv_bfloat16*>(p.st.kbar_op)[so] = __float2bfloat16_rn(sk * inv);
-        reinterpret_cast<__nv_bfloat16*>(p.st.vsum_op)[so] = __float2bfloat16_rn(sv);
         const int pb = nblk & 1;
         sm.ck[pb][c] = sk * inv;
         sm.cv[pb][c] = sv;
@@ -220,6 +236,12 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
       }
       mbar_arrive(&sm.empty[s]);
     }
+    // max |v| of the group: warp maxima through shared memory (red[0][0][0..3] is free here)
+    for (int o = 16; o > 0; o >>= 1) vabs = fmaxf(vabs, __shfl_xor_sync(0xffffffffu, vabs, o));
+    if (lane == 0) sm.red[0][0][warp] = vabs;
+    bar_epi();
+    if (tid == 0)
+      p.vmax[(size_t)bh * nparts + part] = fmaxf(fmaxf(sm.red[0][0][0], sm.red[0][0][1]), fmaxf(sm.red[0][0][2], sm.red[0][0][3]));
     if (ok) ok = !epi_any_failed(!wait_bar(&sm.acc_done, 0, &sm.abort, p.status, p.wait_ns));
     if (ok) {
       tc_fence_after();
@@ -281,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesB; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.empty[s], 129);      // the MMA commit + the 128 threads that copy V out as fp16
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
@@ -350,6 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
   } else {
     const int a = threadIdx.x;                       // H row a == TMEM lane a
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const float vinv = 1.f / p.st.vscale[bh];
+    __half* vop = reinterpret_cast<__half*>(p.st.v_op) + (size_t)bh * p.L * D;
+    __half* vsop = reinterpret_cast<__half*>(p.st.vsum_op);
     float hb[D];
     const float* hbar = p.st.hbar + (size_t)bh * D * D + (size_t)a * D;
 #pragma unroll
@@ -366,11 +391,32 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
       ok = !epi_any_failed(!wait_bar(&sm.acc_full[buf], (t >> 1) & 1, &sm.abort, p.status, p.wait_ns));
       if (!ok) break;
       tc_fence_after();
+      {
+        // fp16 copy of this tile's values, v / vscale: the H_j MMAs of the tile are done, so the stage
+        // has landed and is held until the arrival below; 16-byte chunks, consecutive per thread
+        const uint8_t* vt = sm.v[t % kStagesB];
+        const int rbase = row0 + t * 128;
+        for (int q = a; q < 128 * 16; q += 128) {
+          const int row = q >> 4, c = q & 15;
+          if (rbase + row >= row1) break;
+          const uint4 u = *reinterpret_cast<const uint4*>(vt + (c >> 3) * kHalf + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          uint32_t hw[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const __half2 h2 = __floats2half2_rn(__uint_as_float(w[x] << 16) * vinv, __uint_as_float(w[x] & 0xffff0000u) * vinv);
+            hw[x] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          *reinterpret_cast<uint4*>(vop + (size_t)(rbase + row) * D + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
+        mbar_arrive(&sm.empty[t % kStagesB]);
+      }
       for (int b = 0; b < bpt; ++b) {
         const int j = jb0 + t * bpt + b;
         const bool live = j < jb1;
         const size_t so = ((size_t)bh * p.nb + (live ? j : 0)) * D;
         sm.vs[buf][b][a] = live ? p.st.vsum[so + a] : 0.f;
+        if (live) vsop[so + a] = __float2half_rn(sm.vs[buf][b][a] * vinv);
         const float kb = live ? p.st.kbar[so + a] : 0.f;
         bar_epi();
         float ss = 0.f;
@@ -426,6 +472,7 @@ cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k,
   p.block = g.block;
   p.st = st;
   p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
+  p.vmax = reinterpret_cast<float*>(static_cast<char*>(ws) + vmax_offset(g));
   p.status = static_cast<int*>(ws);
   p.wait_ns = kWaitLimitNs;
   const size_t smem_a = sizeof(SmemA) + 1024, smem_b = sizeof(SmemB) + 1024;
@@ -434,7 +481,7 @@ cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k,
   if ((e = cudaFuncSetAttribute(cov_norm_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
   const int nparts = num_parts(g);
   stats_a_sm100<<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(maps, p);
-  if ((e = launch_hbar_reduce(g, p.partials, nparts, st, stream))) return e;
+  if ((e = launch_hbar_reduce(g, p.partials, nparts, p.vmax, st, stream))) return e;
   cov_norm_sm100<<<dim3((g.nb + kBlocksPerCtaB - 1) / kBlocksPerCtaB, g.BH()), kThreads, smem_b, stream>>>(maps, p);
   return cudaGetLastError();
 }

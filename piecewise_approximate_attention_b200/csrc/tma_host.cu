@@ -26,13 +26,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
                     uint32_t box_rows) {
+  return encode_16bit_3d(map, base, inner, rows, batch, box_rows, false);
+}
+
+bool encode_16bit_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                     uint32_t box_rows, bool fp16) {
   auto fn = encode_fn();
   if (!fn || !base) return false;
   cuuint64_t dims[3] = {inner, rows, batch};
   cuuint64_t strides[2] = {inner * 2, rows * inner * 2};
   cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estride[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
+  const CUresult r = fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

@@ -26,7 +26,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_blocks():
-    assert C.lib().pisa_abi_version() == 1
+    assert C.lib().pisa_abi_version() == 2
     assert C.pisa_num_blocks(32760, 64) == 512
     assert C.pisa_num_blocks(75600, 128) == 591
     assert C.pisa_num_blocks(1, 64) == 1
@@ -55,12 +55,18 @@ def test_stats_bytes_and_carve_are_host_only():
     st = C.PisaStats()
     base = 1 << 20      # never dereferenced: carving is pointer arithmetic
     assert C.lib().pisa_stats_carve(ctypes.byref(sh), base, n1, 1, ctypes.byref(st)) == C.PISA_OK
-    ptrs = [st.qbar, st.kbar, st.vsum, st.hbar, st.M, st.H, st.kbar_op, st.vsum_op, st.hbar_op]
+    ptrs = [st.qbar, st.kbar, st.vsum, st.hbar, st.M, st.H, st.kbar_op, st.vsum_op, st.hbar_op, st.v_op, st.vscale]
     assert all(p and p % 256 == 0 and base <= p < base + n1 for p in ptrs)
     assert len(set(ptrs)) == len(ptrs)
     assert C.lib().pisa_stats_carve(ctypes.byref(sh), base + 16, n1, 1, ctypes.byref(st)) == C.PISA_ERR_INVALID_ARG
     assert C.lib().pisa_stats_carve(ctypes.byref(sh), base, n1 - 1, 1, ctypes.byref(st)) == C.PISA_ERR_INVALID_ARG
     assert C.pisa_workspace_bytes(sh) >= 256 + 2 * 1 * 128 * 128 * 4
+    # fp32 mode needs no tensor-core operand copies
+    f32 = _shape(dtype="fp32")
+    st32 = C.PisaStats()
+    n32 = C.pisa_stats_bytes(f32, False)
+    assert C.lib().pisa_stats_carve(ctypes.byref(f32), base, n32, 0, ctypes.byref(st32)) == C.PISA_OK
+    assert not st32.kbar_op and not st32.v_op and not st32.vscale and n32 < n0
 
 
 @pytest.mark.parametrize("kw,expect", [

@@ -168,6 +168,26 @@ def test_constant_key_blocks_are_dense_on_gpu():
             assert_output(_np(o[0, h]), dense[h], "bf16", what=f"keep {keep} head {h}")
 
 
+def test_value_operand_copy_and_large_values():
+    """The fp16 value operand is v / vscale with vscale a power of two; large values get a larger
+    scale and the output still follows the oracle (o is linear in v)."""
+    w = Workload("vscale", 1, 2, (4, 16, 16), 0, 128, 64, 0.75, 0.5, "bf16", seed=5)
+    q, k, v = make_qkv(w)
+    p, o, _, _ = _run(w, q, k, v)
+    assert torch.equal(p.stats.vscale.cpu(), torch.ones(1, 2))
+    assert torch.equal(p.stats.v_op.cpu(), v.to(torch.float16))
+    big = (v.float() * 3000.0).to(torch.bfloat16)              # max |v| ~ 1.5e4 -> vscale 64
+    p2, o2, _, _ = _run(w, q, k, big)
+    sc = p2.stats.vscale.cpu()
+    assert torch.all(sc == 64.0), sc
+    ref = O.pisa(_np(q), _np(k), _np(big), w.block, w.keep_k, w.lam)
+    for h in range(2):
+        bad, ties = compare_selection(p2.sel[0, h].cpu().numpy(), ref["sel"][0, h], ref["r"][0, h], w.keep_k)
+        assert not bad
+        keep = ~rows_of_blocks(w.seq_len, w.block, ties)
+        assert_output(_np(o2[0, h])[keep], ref["o"][0, h][keep], "bf16", what=f"large values head {h}")
+
+
 def test_order_is_a_permutation():
     w = WORKLOADS["video-dit-small"].with_(heads=2)
     q, k, v = make_qkv(w)

@@ -20,7 +20,7 @@ PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
            "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string",
-           "pisa_precompute_noalloc")
+           "pisa_precompute_noalloc", "pisa_testing_set_attention_fault")
 
 
 class PisaShape(ctypes.Structure):
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "pisa_read_device_error": (i32, [vp, P(i32), vp]),
             "pisa_status_string": (ctypes.c_char_p, [i32]),
             "pisa_precompute_noalloc": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp]),
+            "pisa_testing_set_attention_fault": (i32, [i32, ctypes.c_uint64]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)

@@ -3,11 +3,16 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "pisa_testing.h"
 
 namespace pisa {
 namespace {
 
 constexpr int kMaxBlocks = 4096;
+
+// test-only fault injection (pisa_testing.h)
+int g_test_fault = PISA_TESTING_FAULT_NONE;
+unsigned long long g_test_wait_ns = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -186,8 +191,9 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
         !encode_16bit_3d(&maps.vsum, stats->vsum_op, g.d, g.nb, bh, 128, true) ||
         !encode_bf16_3d(&maps.hbar, stats->hbar_op, g.d, g.d, bh, 128))
       return PISA_ERR_CUDA;
-    return cuda_status(
-        launch_attention_sm100(g, maps, sel, order, keep_k, mode, stats->vscale, o, status, kWaitLimitNs, cs));
+    const unsigned long long wait_ns = g_test_wait_ns ? g_test_wait_ns : kWaitLimitNs;
+    return cuda_status(launch_attention_sm100(g, maps, sel, order, keep_k, mode, stats->vscale, o, status, wait_ns,
+                                              g_test_fault, cs));
   }
   return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status, cs));
 }
@@ -202,6 +208,13 @@ pisa_status pisa_read_device_error(void* ws, int32_t* code, pisa_stream_t stream
   *code = host;
   if (host == 0) return PISA_OK;
   return host == PISA_DEVERR_WAIT_TIMEOUT ? PISA_ERR_DEVICE_TIMEOUT : PISA_ERR_INVALID_ARG;
+}
+
+pisa_status pisa_testing_set_attention_fault(int32_t fault, uint64_t wait_limit_ns) {
+  if (fault != PISA_TESTING_FAULT_NONE && fault != PISA_TESTING_FAULT_SKIP_Q_LOAD) return PISA_ERR_INVALID_ARG;
+  g_test_fault = fault;
+  g_test_wait_ns = wait_limit_ns;
+  return PISA_OK;
 }
 
 const char* pisa_status_string(pisa_status status) {

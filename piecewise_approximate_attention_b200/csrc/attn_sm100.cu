@@ -73,6 +73,7 @@ struct Params {
   float scale_log2;
   float lazy;                // rescale O only when the row max grows by more than this (logit units)
   const float* vscale;       // [B*H] value scale of the fp16 value operands
+  int fault;                 // test-only fault injection (pisa_testing.h); 0 in normal calls
   const int32_t* sel;
   const int32_t* order;
   __nv_bfloat16* o;
@@ -229,12 +230,14 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
-      mbar_expect_tx(&sm.bar_q, kTileBytes);
-      tma_load_3d(sm.q, &maps.q, &sm.bar_q, 0, qa * p.block, bh);
-      tma_load_3d(sm.q + kHalf, &maps.q, &sm.bar_q, 64, qa * p.block, bh);
-      if (pair) {
-        tma_load_3d(sm.q + 64 * 128, &maps.q, &sm.bar_q, 0, qb * p.block, bh);
-        tma_load_3d(sm.q + kHalf + 64 * 128, &maps.q, &sm.bar_q, 64, qb * p.block, bh);
+      if (p.fault != 1) {      // fault 1 (tests only): never load Q, so the MMA warp's wait runs out
+        mbar_expect_tx(&sm.bar_q, kTileBytes);
+        tma_load_3d(sm.q, &maps.q, &sm.bar_q, 0, qa * p.block, bh);
+        tma_load_3d(sm.q + kHalf, &maps.q, &sm.bar_q, 64, qa * p.block, bh);
+        if (pair) {
+          tma_load_3d(sm.q + 64 * 128, &maps.q, &sm.bar_q, 0, qb * p.block, bh);
+          tma_load_3d(sm.q + kHalf + 64 * 128, &maps.q, &sm.bar_q, 64, qb * p.block, bh);
+        }
       }
       UnionIter it;
       int issued_k = 0, issued_v = 0;
@@ -539,7 +542,7 @@ size_t attention_sm100_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
                                    int keep_k, int mode, const float* vscale, void* o, int* status,
-                                   unsigned long long wait_ns, cudaStream_t stream) {
+                                   unsigned long long wait_ns, int fault, cudaStream_t stream) {
   Params p;
   p.L = g.L;
   p.nb = g.nb;
@@ -550,6 +553,7 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
   p.scale_log2 = g.scale * 1.4426950408889634f;
   p.lazy = kLazyLog2 / p.scale_log2;
   p.vscale = vscale;
+  p.fault = fault;
   p.sel = sel;
   p.order = order;
   p.o = static_cast<__nv_bfloat16*>(o);

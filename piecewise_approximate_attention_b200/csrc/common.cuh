@@ -75,7 +75,7 @@ cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float 
                          int32_t* order, float* scores, cudaStream_t stream);
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
                                    int keep_k, int mode, const float* vscale, void* o, int* status,
-                                   unsigned long long wait_ns, cudaStream_t stream);
+                                   unsigned long long wait_ns, int fault, cudaStream_t stream);
 cudaError_t launch_attention_simt(const Dims& g, const void* q, const void* k, const void* v,
                                   const pisa_stats& st, const int32_t* sel, int keep_k, int mode,
                                   void* o, int* status, cudaStream_t stream);

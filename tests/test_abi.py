@@ -12,14 +12,15 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "pisa.h")).read()
+    import glob
+    src = "".join(open(f).read() for f in glob.glob(os.path.join(ROOT, "include", "*.h")))
     return sorted(set(re.findall(r"PISA_API\s+[\w\s\*]*?\b(pisa_\w+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_symbol():
     lib = C.lib()
     names = _declared()
-    assert len(names) >= 10
+    assert len(names) >= 12
     assert set(names) == set(C.SYMBOLS)
     for n in names:
         assert hasattr(lib, n), n
@@ -134,3 +135,8 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(C, "_LIB_PATH", "/nonexistent/libpisa_b200.so")
     with pytest.raises(RuntimeError, match="not built"):
         C.lib()
+
+
+def test_testing_hook_rejects_unknown_fault():
+    assert C.lib().pisa_testing_set_attention_fault(7, 0) == C.PISA_ERR_INVALID_ARG
+    assert C.lib().pisa_testing_set_attention_fault(0, 0) == C.PISA_OK

@@ -1,0 +1,51 @@
+"""Failure detection on the GPU without a fault: a bounded wait that runs out is reported.
+
+The test-only hook makes the attention kernel skip its query-tile load, so the MMA warp's wait for
+it can never complete.  The kernel must record PISA_DEVERR_WAIT_TIMEOUT in the workspace status
+word within its (shortened) wait limit, drain its own work, free its tensor memory and return; the
+next call on the same context must then run normally and match the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import pisa_oracle as O
+from piecewise_approximate_attention_b200 import _lib as C
+from piecewise_approximate_attention_b200.runtime import Pisa
+from piecewise_approximate_attention_b200.workloads import Workload, make_qkv
+from tests.parity import assert_output, compare_selection, rows_of_blocks
+
+pytestmark = pytest.mark.gpu
+
+SKIP_Q_LOAD = 1
+WAIT_NS = 20_000_000          # 20 ms instead of the default 2 s
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    w = Workload("fault", 1, 1, (2, 16, 16), 0, 128, 128, 0.5, 0.5, "bf16", seed=2)
+    q, k, v = make_qkv(w)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    p = Pisa(1, 1, w.seq_len, 128, w.block, w.keep_k, w.lam, "bf16", 1.0, "cuda")
+    p.precompute(qd, kd, vd)
+    p.route()
+    torch.cuda.synchronize()
+    assert p.device_error() == (C.PISA_OK, 0)
+    o = torch.zeros_like(qd)
+    assert C.lib().pisa_testing_set_attention_fault(SKIP_Q_LOAD, WAIT_NS) == C.PISA_OK
+    try:
+        p.attention(qd, kd, vd, o)
+        torch.cuda.synchronize()
+    finally:
+        assert C.lib().pisa_testing_set_attention_fault(0, 0) == C.PISA_OK
+    assert p.device_error() == (C.PISA_ERR_DEVICE_TIMEOUT, C.PISA_DEVERR_WAIT_TIMEOUT)
+    assert p.device_error() == (C.PISA_OK, 0)          # read clears the status word
+    # the context is intact: a normal call works and is correct
+    o2 = torch.empty_like(qd)
+    p.attention(qd, kd, vd, o2)
+    torch.cuda.synchronize()
+    assert p.device_error() == (C.PISA_OK, 0)
+    ref = O.pisa(q.double().numpy(), k.double().numpy(), v.double().numpy(), w.block, w.keep_k, w.lam)
+    bad, ties = compare_selection(p.sel[0, 0].cpu().numpy(), ref["sel"][0, 0], ref["r"][0, 0], w.keep_k)
+    assert not bad
+    keep = ~rows_of_blocks(w.seq_len, w.block, ties)
+    assert_output(o2[0, 0].double().cpu().numpy()[keep], ref["o"][0, 0][keep], "bf16", what="after timeout")

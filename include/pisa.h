@@ -57,8 +57,13 @@ typedef enum {
 typedef enum { PISA_BF16 = 0, PISA_FP32 = 1 } pisa_dtype;
 
 /* PISA_MODE_EXACT_ONLY drops U_i entirely (the keep-or-drop sparse attention the method is
- * compared against, §1 문제 정의); it needs keep_k >= 1. */
-typedef enum { PISA_MODE_PISA = 0, PISA_MODE_EXACT_ONLY = 1 } pisa_mode;
+ * compared against, §1 문제 정의); it needs keep_k >= 1.
+ * PISA_MODE_PER_BLOCK replaces the global first-order term by each unselected block's own one,
+ *     N_t += s sum_{j in U_i} alpha_{t,j} (q_t H_j)      instead of   s (q_t Hbar) sum_{j in U_i} alpha_{t,j},
+ * the per-block form that §2 핵심 알고리즘 sets aside because it loads one d x d matrix per block.
+ * It is a diagnostic of what the shared Hbar gives up; it needs the per-block matrices in the
+ * stats (carved with with_H != 0 and written by pisa_precompute). */
+typedef enum { PISA_MODE_PISA = 0, PISA_MODE_EXACT_ONLY = 1, PISA_MODE_PER_BLOCK = 2 } pisa_mode;
 
 typedef struct {
   int32_t batch;          /* B >= 1 */
@@ -88,6 +93,8 @@ typedef struct {
   void*  hbar_op;  /* bf16 [B,H,d,d]   softmax_scale * Hbar^T, i.e. hbar_op[c][a]              */
   void*  v_op;     /* fp16 [B,H,L,d]   v / vscale (exact for every bf16 value in fp16 range)   */
   float* vscale;   /* [B,H]            power of two >= max|v| / 256 (1 when max|v| <= 256)     */
+  void*  hdiff_op; /* nullable bf16 [B,H,nb,d,d]: softmax_scale * (H_j - Hbar), row a = key dim;
+                    * written only when non-null (PISA_BF16 and with_H); PISA_MODE_PER_BLOCK reads it */
 } pisa_stats;
 
 /* ABI revision of this header. */
@@ -97,7 +104,8 @@ PISA_API int32_t pisa_abi_version(void);
 PISA_API int32_t pisa_num_blocks(int32_t seq_len, int32_t block);
 
 /* Bytes of one contiguous buffer that pisa_stats_carve can split into every pisa_stats array
- * (H included when with_H != 0; the operand copies only for PISA_BF16).  0 if the shape is invalid. */
+ * (H, and for PISA_BF16 hdiff_op, included when with_H != 0; the operand copies only for
+ * PISA_BF16).  0 if the shape is invalid. */
 PISA_API size_t pisa_stats_bytes(const pisa_shape* shape, int32_t with_H);
 
 /* Host-only pointer arithmetic: fills *out with 256-byte-aligned sub-ranges of [base, base+bytes).
@@ -106,7 +114,8 @@ PISA_API pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_
                              pisa_stats* out);
 
 /* Device scratch bytes needed by pisa_precompute and pisa_attention for this shape (the first 256
- * bytes hold the device status word read by pisa_read_device_error). */
+ * bytes hold the device status word read by pisa_read_device_error; the rest is transient scratch:
+ * partial sums in pisa_precompute, per-row softmax offsets in PISA_MODE_PER_BLOCK). */
 PISA_API size_t pisa_workspace_bytes(const pisa_shape* shape);
 
 /* Pre-computation (§2 하드웨어 구현, step 1; zeroth-order and global first-order bullets of
@@ -152,7 +161,12 @@ PISA_API pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats
  * stages 1-3: exact selected blocks, zeroth-order scan of the other blocks, global first-order
  * correction).  sel as written by pisa_route (ascending, distinct, < nb; checked on the device,
  * a bad entry sets the status word).  order: nullable, as written by pisa_route; null means
- * 0, 1, ..., nb-1.  o: [B,H,L,d] of dtype.  mode: pisa_mode.  ws as for pisa_precompute. */
+ * 0, 1, ..., nb-1.  o: [B,H,L,d] of dtype.  mode: pisa_mode.  ws as for pisa_precompute.
+ * PISA_MODE_PER_BLOCK needs stats->hdiff_op (PISA_BF16) or stats->H (PISA_FP32) non-null and
+ * written by the pisa_precompute call that wrote the other stats; otherwise PISA_ERR_INVALID_ARG.
+ * On the bf16 path it is two launches: the attention kernel, which also leaves each row's softmax
+ * offset and 1/D_t in ws, then a tensor-core kernel that adds s sum_j alpha_{t,j} q_t (H_j - Hbar)
+ * / D_t to o over the unselected blocks (o is read back in bf16 and rounded once more). */
 PISA_API pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k, const void* v,
                            const pisa_stats* stats, const int32_t* sel, const int32_t* order,
                            int32_t keep_k, int32_t mode, void* o, void* ws, size_t ws_bytes,

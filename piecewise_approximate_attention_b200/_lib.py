@@ -15,7 +15,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "lib
 
 PISA_OK, PISA_ERR_INVALID_ARG, PISA_ERR_UNSUPPORTED, PISA_ERR_CUDA, PISA_ERR_DEVICE_TIMEOUT = range(5)
 PISA_BF16, PISA_FP32 = 0, 1
-PISA_MODE_PISA, PISA_MODE_EXACT_ONLY = 0, 1
+PISA_MODE_PISA, PISA_MODE_EXACT_ONLY, PISA_MODE_PER_BLOCK = 0, 1, 2
 PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
@@ -31,7 +31,8 @@ class PisaShape(ctypes.Structure):
 
 class PisaStats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("qbar", "kbar", "vsum", "hbar", "M", "H", "kbar_op", "vsum_op", "hbar_op", "v_op", "vscale")]
+                ("qbar", "kbar", "vsum", "hbar", "M", "H", "kbar_op", "vsum_op", "hbar_op", "v_op", "vscale",
+                 "hdiff_op")]
 
 
 class PisaError(RuntimeError):
@@ -137,6 +138,7 @@ class Stats:
     hbar_op: object
     v_op: object
     vscale: object
+    hdiff_op: Optional[object]
 
 
 def alloc_stats(shape: PisaShape, device, with_H: bool = False) -> Stats:
@@ -167,7 +169,8 @@ def alloc_stats(shape: PisaShape, device, with_H: bool = False) -> Stats:
                  view(st.vsum, f32, (B, H, nb, d)), view(st.hbar, f32, (B, H, d, d)), view(st.M, f32, (B, H, nb)),
                  view(st.H, f32, (B, H, nb, d, d)), view(st.kbar_op, bf, (B, H, nb, d)),
                  view(st.vsum_op, f16, (B, H, nb, d)), view(st.hbar_op, bf, (B, H, d, d)),
-                 view(st.v_op, f16, (B, H, shape.seq_len, d)), view(st.vscale, f32, (B, H)))
+                 view(st.v_op, f16, (B, H, shape.seq_len, d)), view(st.vscale, f32, (B, H)),
+                 view(st.hdiff_op, bf, (B, H, nb, d, d)))
 
 
 def alloc_workspace(shape: PisaShape, device):

@@ -46,7 +46,7 @@ pisa_status check_stats(const Dims& g, const pisa_stats* st, bool need_ops) {
   const void* req[] = {st->qbar, st->kbar, st->vsum, st->hbar, st->M};
   for (const void* p : req)
     if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
-  if (st->H && !aligned16(st->H)) return PISA_ERR_INVALID_ARG;
+  if ((st->H && !aligned16(st->H)) || (st->hdiff_op && !aligned16(st->hdiff_op))) return PISA_ERR_INVALID_ARG;
   if (need_ops && g.dtype == PISA_BF16) {
     const void* ops[] = {st->kbar_op, st->vsum_op, st->hbar_op, st->v_op, st->vscale};
     for (const void* p : ops)
@@ -59,7 +59,7 @@ pisa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PISA_OK : PIS
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-constexpr int kStatsArrays = 11;
+constexpr int kStatsArrays = 12;
 
 // Sizes of the stats arrays in carve order.
 void stats_sizes(const Dims& g, int with_H, size_t out[kStatsArrays]) {
@@ -76,6 +76,7 @@ void stats_sizes(const Dims& g, int with_H, size_t out[kStatsArrays]) {
   out[8] = ops ? bh * d * d * 2 : 0;   // hbar_op
   out[9] = ops ? bh * (size_t)g.L * d * 2 : 0;   // v_op
   out[10] = ops ? bh * 4 : 0;          // vscale
+  out[11] = (ops && with_H) ? bh * nb * d * d * 2 : 0;   // hdiff_op
 }
 
 }  // namespace
@@ -85,7 +86,7 @@ using namespace pisa;
 
 extern "C" {
 
-int32_t pisa_abi_version(void) { return 2; }
+int32_t pisa_abi_version(void) { return 3; }
 
 int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
   if (seq_len < 1 || block < 1) return -1;
@@ -128,6 +129,7 @@ pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, 
   st.hbar_op = ptr[8];
   st.v_op = ptr[9];
   st.vscale = static_cast<float*>(ptr[10]);
+  st.hdiff_op = ptr[11];
   *out = st;
   return PISA_OK;
 }
@@ -135,7 +137,9 @@ pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, 
 size_t pisa_workspace_bytes(const pisa_shape* shape) {
   Dims g;
   if (check_shape(shape, &g) != PISA_OK) return 0;
-  return kStatusBytes + round_up(partials_bytes(g), 256) + round_up(vmax_bytes(g), 256);
+  const size_t pre = round_up(partials_bytes(g), 256) + round_up(vmax_bytes(g), 256);
+  const size_t rows = round_up(rowstats_bytes(g), 256);
+  return kStatusBytes + (pre > rows ? pre : rows);
 }
 
 pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
@@ -174,11 +178,13 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
   if (!q || !k || !v || !o || !ws || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       !aligned16(ws))
     return PISA_ERR_INVALID_ARG;
-  if (mode != PISA_MODE_PISA && mode != PISA_MODE_EXACT_ONLY) return PISA_ERR_INVALID_ARG;
+  if (mode != PISA_MODE_PISA && mode != PISA_MODE_EXACT_ONLY && mode != PISA_MODE_PER_BLOCK)
+    return PISA_ERR_INVALID_ARG;
   if (keep_k < 0 || keep_k > g.nb || (mode == PISA_MODE_EXACT_ONLY && keep_k < 1)) return PISA_ERR_INVALID_ARG;
   if (keep_k > 0 && (!sel || !aligned16(sel))) return PISA_ERR_INVALID_ARG;
   if (order && !aligned16(order)) return PISA_ERR_INVALID_ARG;
   if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
+  if (mode == PISA_MODE_PER_BLOCK && !(g.dtype == PISA_BF16 ? stats->hdiff_op : stats->H)) return PISA_ERR_INVALID_ARG;
   if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   int* status = static_cast<int*>(ws);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -192,8 +198,16 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
         !encode_bf16_3d(&maps.hbar, stats->hbar_op, g.d, g.d, bh, 128))
       return PISA_ERR_CUDA;
     const unsigned long long wait_ns = g_test_wait_ns ? g_test_wait_ns : kWaitLimitNs;
-    return cuda_status(launch_attention_sm100(g, maps, sel, order, keep_k, mode, stats->vscale, o, status, wait_ns,
-                                              g_test_fault, cs));
+    // per-block mode: the attention kernel runs in PISA mode and leaves each row's softmax offset and
+    // 1/D_t behind; the second kernel adds the per-block minus global first-order difference
+    const bool per_block = mode == PISA_MODE_PER_BLOCK && keep_k < g.nb;
+    float2* rows = per_block ? reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes) : nullptr;
+    cudaError_t e = launch_attention_sm100(g, maps, sel, order, keep_k, mode == PISA_MODE_EXACT_ONLY ? mode : PISA_MODE_PISA,
+                                           stats->vscale, o, rows, status, wait_ns, g_test_fault, cs);
+    if (e != cudaSuccess || !per_block) return cuda_status(e);
+    CUtensorMap hmap;
+    if (!encode_bf16_3d(&hmap, stats->hdiff_op, g.d, (uint64_t)g.nb * g.d, bh, 128)) return PISA_ERR_CUDA;
+    return cuda_status(launch_perblock_sm100(g, maps, hmap, sel, order, keep_k, rows, o, status, wait_ns, cs));
   }
   return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status, cs));
 }

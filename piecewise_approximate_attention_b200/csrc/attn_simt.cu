@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(128) attn_simt(const T* __restrict__ q, const 
     }
   }
   // stage 2: zeroth-order scan over the centroids of the unselected blocks
-  const bool approx = mode == PISA_MODE_PISA && nsel < nb;
+  const bool approx = (mode == PISA_MODE_PISA || mode == PISA_MODE_PER_BLOCK) && nsel < nb;
   if (approx) {
     const size_t so = (size_t)bh * nb * D;
     for (int j0 = 0; j0 < nb; j0 += kTile) {
@@ -135,8 +135,39 @@ __global__ void __launch_bounds__(128) attn_simt(const T* __restrict__ q, const 
       process_tile(ncols, true, mask);
     }
   }
+  // stage 3 (per-block variant): N += s * alpha_tj * (q_t H_j) for every j in U_i, H_j streamed
+  // through the key tile; m is final after stage 2, so alpha_tj = e^{s q_t.kbar_j - m}
+  if (approx && mode == PISA_MODE_PER_BLOCK) {
+    const size_t so = (size_t)bh * nb * D;
+    for (int j = 0; j < nb; ++j) {
+      if ((sm.selbits[j >> 5] >> (j & 31)) & 1u) continue;
+      __syncthreads();
+      for (int a = t; a < D; a += blockDim.x) sm.vt[0][a] = st.kbar[so + (size_t)j * D + a];
+      __syncthreads();
+      float f = 0.f;
+      if (row_ok) {
+        float dot = 0.f;
+#pragma unroll 16
+        for (int a = 0; a < D; ++a) dot = fmaf(sm.q[t][a], sm.vt[0][a], dot);
+        f = scale * expf(scale * dot - m);
+      }
+      const float* hj = st.H + ((size_t)bh * nb + j) * D * D;
+      for (int a0 = 0; a0 < D; a0 += kTile) {
+        __syncthreads();
+        for (int idx = t; idx < kTile * D; idx += blockDim.x) sm.kt[idx / D][idx % D] = hj[(size_t)a0 * D + idx];
+        __syncthreads();
+        if (row_ok) {
+          for (int a = 0; a < kTile; ++a) {
+            const float fa = f * sm.q[t][a0 + a];
+#pragma unroll
+            for (int c = 0; c < D; ++c) acc[c] = fmaf(fa, sm.kt[a][c], acc[c]);
+          }
+        }
+      }
+    }
+  }
   // stage 3: first-order correction  N += s * A * (q_t Hbar), Hbar streamed through the key tile
-  if (approx) {
+  else if (approx) {
     const float* hb = st.hbar + (size_t)bh * D * D;
     for (int a0 = 0; a0 < D; a0 += kTile) {
       __syncthreads();

@@ -77,6 +77,7 @@ struct Params {
   const int32_t* sel;
   const int32_t* order;
   __nv_bfloat16* o;
+  float2* rowstats;          // nullable [B*H][L]: (softmax offset m*s*log2(e), 1/D_t) per row
   int* status;
   unsigned long long wait_ns;
 };
@@ -504,7 +505,9 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l, vsc = p.vscale[bh];
-      __nv_bfloat16* orow = p.o + ((size_t)bh * p.L + (size_t)myq * p.block + rloc) * D;
+      const size_t grow_idx = (size_t)bh * p.L + (size_t)myq * p.block + rloc;
+      __nv_bfloat16* orow = p.o + grow_idx * D;
+      if (p.rowstats && row_valid) p.rowstats[grow_idx] = make_float2(m == -INFINITY ? 0.f : m * p.scale_log2, inv);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float ov[32], cv[32];
@@ -541,8 +544,8 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
 size_t attention_sm100_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
-                                   int keep_k, int mode, const float* vscale, void* o, int* status,
-                                   unsigned long long wait_ns, int fault, cudaStream_t stream) {
+                                   int keep_k, int mode, const float* vscale, void* o, float2* rowstats,
+                                   int* status, unsigned long long wait_ns, int fault, cudaStream_t stream) {
   Params p;
   p.L = g.L;
   p.nb = g.nb;
@@ -557,6 +560,7 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
   p.sel = sel;
   p.order = order;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.rowstats = rowstats;
   p.status = status;
   p.wait_ns = wait_ns;
   const size_t smem = attention_sm100_smem_bytes();

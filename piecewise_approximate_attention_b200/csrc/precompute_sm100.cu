@@ -92,6 +92,7 @@ struct KVMaps {
 
 struct PreParams {
   int L, nb, block;
+  float scale;               // softmax scale (folded into the per-block first-order operand copy)
   pisa_stats st;
   float* partials;
   float* vmax;               // [BH][nparts] max |v| per group (pass A)
@@ -421,22 +422,34 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
         bar_epi();
         float ss = 0.f;
         float* Hout = (live && p.st.H) ? p.st.H + ((size_t)bh * p.nb + j) * D * D + (size_t)a * D : nullptr;
+        __nv_bfloat16* Dout = (live && p.st.hdiff_op)
+                                  ? static_cast<__nv_bfloat16*>(p.st.hdiff_op) + ((size_t)bh * p.nb + j) * D * D + (size_t)a * D
+                                  : nullptr;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           float h[32];
           tmem_ld32(trow + (uint32_t)(buf * 256 + b * 128 + 32 * ch), h);
           tmem_ld_wait();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int c = 32 * ch + x;
-            h[x] = fmaf(-kb, sm.vs[buf][b][c], h[x]);
-            const float dl = h[x] - hb[c];
-            ss = fmaf(dl, dl, ss);
-          }
+          for (int x = 0; x < 32; ++x) h[x] = fmaf(-kb, sm.vs[buf][b][32 * ch + x], h[x]);
           if (Hout) {
 #pragma unroll
             for (int x = 0; x < 32; x += 4)
               *reinterpret_cast<float4*>(Hout + 32 * ch + x) = make_float4(h[x], h[x + 1], h[x + 2], h[x + 3]);
+          }
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            h[x] -= hb[32 * ch + x];      // H_j - Hbar
+            ss = fmaf(h[x], h[x], ss);
+          }
+          if (Dout) {
+            // operand copy of the per-block first-order difference: s (H_j - Hbar), row a, bf16
+            uint32_t pk[16];
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) pk[x >> 1] = pack_bf16x2(p.scale * h[x], p.scale * h[x + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(Dout + 32 * ch);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
           }
         }
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -470,6 +483,7 @@ cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k,
   p.L = g.L;
   p.nb = g.nb;
   p.block = g.block;
+  p.scale = g.scale;
   p.st = st;
   p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
   p.vmax = reinterpret_cast<float*>(static_cast<char*>(ws) + vmax_offset(g));

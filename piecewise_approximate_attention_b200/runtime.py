@@ -26,6 +26,9 @@ class Pisa:
         self.nb = C.pisa_num_blocks(seq_len, block)
         self.device = torch.device(device)
         self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self._torch_f32 = torch.float32
+        if mode == C.PISA_MODE_PER_BLOCK:
+            with_H = True         # the per-block first-order matrices live in the stats
         self.stats = C.alloc_stats(self.shape, self.device, with_H)
         self.ws = C.alloc_workspace(self.shape, self.device)
         self.sel = torch.empty((batch, heads, self.nb, max(keep_k, 1)), dtype=torch.int32, device=self.device)
@@ -53,8 +56,11 @@ class Pisa:
         return o
 
     def launches_per_step(self) -> int:
-        """Kernels one __call__ enqueues: pre-compute 3, routing 1 (+1 pairing), attention 1."""
-        return 3 + 1 + (1 if self.order is not None else 0) + 1
+        """Kernels one __call__ enqueues: pre-compute 3, routing 1 (+1 pairing), attention 1 (+1 for
+        the per-block first-order kernel on the bf16 path)."""
+        extra = 1 if (self.mode == C.PISA_MODE_PER_BLOCK and self.tdtype != self._torch_f32 and
+                      self.keep_k < self.nb) else 0
+        return 3 + 1 + (1 if self.order is not None else 0) + 1 + extra
 
     def device_error(self, stream=None):
         return C.pisa_read_device_error(self.ws, stream)

@@ -27,7 +27,8 @@ from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "keep_from_sparsity", "make_head", "make_qkv", "to_dtype"]
+__all__ = ["Workload", "WORKLOADS", "keep_from_sparsity", "make_head", "make_qkv", "to_dtype",
+           "make_block_structured"]
 
 
 def keep_from_sparsity(nb: int, sparsity: float) -> int:
@@ -145,3 +146,25 @@ def make_qkv(w: Workload, heads: Optional[Sequence[int]] = None, seed: Optional[
             for t, arr in zip(out, make_head(w, b, h, seed)):
                 t[b, i].copy_(to_dtype(arr, w.dtype))
     return out[0], out[1], out[2]
+
+
+def make_block_structured(seq_len: int, head_dim: int, block: int, dtype: str, seed: int = 0,
+                          spread: float = 0.5, qscale: float = 1.5):
+    """CPU torch tensors q, k, v [1, 1, L, d] whose key blocks carry strong, block-specific
+    key/value covariance, so that each block's first-order matrix differs markedly from their mean.
+
+    From ``default_rng([seed, 1000003])``: per block j a centre c_j ~ 0.6 N(0,1)^d and a sign
+    s_j in {-1, +1}; per token n of block j a deviation e_n ~ N(0,1)^d; then
+        k_n = c_j + spread * e_n,    v_n = 0.5 N(0,1)^d + s_j * e_n,    q_n = qscale * N(0,1)^d / sqrt(d).
+    """
+    rng = np.random.default_rng([seed, 1000003])
+    L, d = seq_len, head_dim
+    nb = -(-L // block)
+    centre = 0.6 * rng.standard_normal((nb, d))
+    sign = rng.choice([-1.0, 1.0], size=nb)
+    dev = rng.standard_normal((L, d))
+    owner = np.arange(L) // block
+    k = centre[owner] + spread * dev
+    v = 0.5 * rng.standard_normal((L, d)) + sign[owner][:, None] * dev
+    q = qscale * rng.standard_normal((L, d)) / math.sqrt(d)
+    return tuple(to_dtype(x.astype(np.float32), dtype)[None, None] for x in (q, k, v))

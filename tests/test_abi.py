@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_blocks():
-    assert C.lib().pisa_abi_version() == 2
+    assert C.lib().pisa_abi_version() == 3
     assert C.pisa_num_blocks(32760, 64) == 512
     assert C.pisa_num_blocks(75600, 128) == 591
     assert C.pisa_num_blocks(1, 64) == 1
@@ -52,11 +52,12 @@ def test_stats_bytes_and_carve_are_host_only():
     n0 = C.pisa_stats_bytes(sh, False)
     n1 = C.pisa_stats_bytes(sh, True)
     nb = 16
-    assert n1 - n0 >= 2 * nb * 128 * 128 * 4
+    assert n1 - n0 >= nb * 128 * 128 * (4 + 2)       # H (fp32) and its bf16 difference copy
     st = C.PisaStats()
     base = 1 << 20      # never dereferenced: carving is pointer arithmetic
     assert C.lib().pisa_stats_carve(ctypes.byref(sh), base, n1, 1, ctypes.byref(st)) == C.PISA_OK
-    ptrs = [st.qbar, st.kbar, st.vsum, st.hbar, st.M, st.H, st.kbar_op, st.vsum_op, st.hbar_op, st.v_op, st.vscale]
+    ptrs = [st.qbar, st.kbar, st.vsum, st.hbar, st.M, st.H, st.kbar_op, st.vsum_op, st.hbar_op, st.v_op, st.vscale,
+            st.hdiff_op]
     assert all(p and p % 256 == 0 and base <= p < base + n1 for p in ptrs)
     assert len(set(ptrs)) == len(ptrs)
     assert C.lib().pisa_stats_carve(ctypes.byref(sh), base + 16, n1, 1, ctypes.byref(st)) == C.PISA_ERR_INVALID_ARG
@@ -68,6 +69,13 @@ def test_stats_bytes_and_carve_are_host_only():
     n32 = C.pisa_stats_bytes(f32, False)
     assert C.lib().pisa_stats_carve(ctypes.byref(f32), base, n32, 0, ctypes.byref(st32)) == C.PISA_OK
     assert not st32.kbar_op and not st32.v_op and not st32.vscale and n32 < n0
+    # without H there is no per-block operand copy; fp32 keeps H but has no operand copies
+    st0 = C.PisaStats()
+    assert C.lib().pisa_stats_carve(ctypes.byref(sh), base, n0, 0, ctypes.byref(st0)) == C.PISA_OK
+    assert not st0.H and not st0.hdiff_op
+    n32h = C.pisa_stats_bytes(f32, True)
+    assert C.lib().pisa_stats_carve(ctypes.byref(f32), base, n32h, 1, ctypes.byref(st32)) == C.PISA_OK
+    assert st32.H and not st32.hdiff_op
 
 
 @pytest.mark.parametrize("kw,expect", [
@@ -120,7 +128,10 @@ def test_invalid_arguments_rejected_without_launch():
     # attention arguments
     att = lambda keep, mode, sel=P, o=P, wsb=ws: L.pisa_attention(bs, P, P, P, ctypes.byref(st), sel, None, keep,
                                                                   mode, o, P, wsb, None)
-    assert att(4, 2) == C.PISA_ERR_INVALID_ARG
+    assert att(4, 3) == C.PISA_ERR_INVALID_ARG
+    assert att(4, -1) == C.PISA_ERR_INVALID_ARG
+    # the per-block first-order mode needs the per-block operand copy in the stats
+    assert att(4, C.PISA_MODE_PER_BLOCK) == C.PISA_ERR_INVALID_ARG
     assert att(0, C.PISA_MODE_EXACT_ONLY) == C.PISA_ERR_INVALID_ARG
     assert att(17, C.PISA_MODE_PISA) == C.PISA_ERR_INVALID_ARG
     assert att(4, C.PISA_MODE_PISA, sel=None) == C.PISA_ERR_INVALID_ARG

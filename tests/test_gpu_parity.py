@@ -128,24 +128,33 @@ EDGE = [
     ("bf16", (10, 10, 10), 0, 128, 2, 0.5, C.PISA_MODE_PISA),
     ("bf16", (1, 19, 20), 9, 64, 3, 0.5, C.PISA_MODE_PISA),
     ("bf16", (4, 16, 16), 0, 64, 5, 3.0, C.PISA_MODE_PISA),
+    ("bf16", (10, 10, 10), 0, 64, 3, 0.5, C.PISA_MODE_PER_BLOCK),
+    ("bf16", (10, 10, 10), 0, 64, 0, 0.5, C.PISA_MODE_PER_BLOCK),
+    ("bf16", (10, 10, 10), 0, 64, 16, 0.5, C.PISA_MODE_PER_BLOCK),
+    ("bf16", (2, 5, 5), 0, 64, 1, 0.5, C.PISA_MODE_PER_BLOCK),
+    ("bf16", (1, 19, 20), 9, 128, 2, 0.5, C.PISA_MODE_PER_BLOCK),
     ("fp32", (10, 10, 10), 0, 64, 3, 0.5, C.PISA_MODE_PISA),
     ("fp32", (1, 19, 20), 9, 128, 2, 1.0, C.PISA_MODE_EXACT_ONLY),
     ("fp32", (2, 5, 5), 0, 64, 0, 0.5, C.PISA_MODE_PISA),
+    ("fp32", (1, 19, 20), 9, 128, 2, 0.5, C.PISA_MODE_PER_BLOCK),
+    ("fp32", (2, 5, 5), 0, 64, 0, 0.5, C.PISA_MODE_PER_BLOCK),
 ]
+# the bf16 tensor-core path is built for head_dim 128 only; fp32 runs both head sizes
+EDGE_CASES = [(c, hd) for c in EDGE for hd in ((64, 128) if c[0] == "fp32" else (128,))]
+_MODE_NAME = {C.PISA_MODE_PISA: "pisa", C.PISA_MODE_EXACT_ONLY: "exact", C.PISA_MODE_PER_BLOCK: "perblock"}
 
 
-@pytest.mark.parametrize("case", EDGE, ids=[f"{c[0]}-L{c[1][0]*c[1][1]*c[1][2]+c[2]}-b{c[3]}-k{c[4]}-m{c[6]}"
-                                            for c in EDGE])
-@pytest.mark.parametrize("head_dim", [64, 128])
+@pytest.mark.parametrize("case,head_dim", EDGE_CASES,
+                         ids=[f"{c[0]}-d{hd}-L{c[1][0]*c[1][1]*c[1][2]+c[2]}-b{c[3]}-k{c[4]}-{_MODE_NAME[c[6]]}"
+                              for c, hd in EDGE_CASES])
 def test_edge_cases(case, head_dim):
     dtype, grid, text, block, keep_k, lam, mode = case
-    if dtype == "bf16" and head_dim != 128:
-        pytest.skip("bf16 path is built for head_dim 128")
     w = Workload("edge", 2, 2, grid, text, head_dim, block, 0.5, lam, dtype, seed=7)
     q, k, v = make_qkv(w)
     p, o, scores, qkv = _run(w, q, k, v, keep_k=keep_k, lam=lam, mode=mode, scale=0.9)
-    md = "pisa" if mode == C.PISA_MODE_PISA else "exact_only"
-    ref = O.pisa(_np(q), _np(k), _np(v), block, keep_k, lam, 0.9, mode=md)
+    md = "exact_only" if mode == C.PISA_MODE_EXACT_ONLY else "pisa"
+    fo = "per_block" if mode == C.PISA_MODE_PER_BLOCK else "global"
+    ref = O.pisa(_np(q), _np(k), _np(v), block, keep_k, lam, 0.9, mode=md, first_order=fo)
     for b in range(2):
         for h in range(2):
             bad, ties = compare_selection(p.sel[b, h].cpu().numpy()[:, :keep_k], ref["sel"][b, h], ref["r"][b, h],

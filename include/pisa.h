@@ -118,6 +118,12 @@ PISA_API pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_
  * partial sums in pisa_precompute, per-row softmax offsets in PISA_MODE_PER_BLOCK). */
 PISA_API size_t pisa_workspace_bytes(const pisa_shape* shape);
 
+/* Device scratch bytes that pisa_attention needs in PISA_MODE_PER_BLOCK (never less than
+ * pisa_workspace_bytes): the status word, each row's softmax offset and 1/D_t, and the attention
+ * output in fp32, B*H*L*d*4 bytes, so that o is rounded to bf16 only once.  0 if the shape is
+ * invalid. */
+PISA_API size_t pisa_perblock_workspace_bytes(const pisa_shape* shape);
+
 /* Pre-computation (§2 하드웨어 구현, step 1; zeroth-order and global first-order bullets of
  * 핵심 알고리즘; M_j from 공분산 인식 라우팅): from q, k, v writes every array of *stats.
  * ws: device scratch of at least pisa_workspace_bytes(shape).  Its first 256 bytes hold the device
@@ -163,10 +169,11 @@ PISA_API pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats
  * a bad entry sets the status word).  order: nullable, as written by pisa_route; null means
  * 0, 1, ..., nb-1.  o: [B,H,L,d] of dtype.  mode: pisa_mode.  ws as for pisa_precompute.
  * PISA_MODE_PER_BLOCK needs stats->hdiff_op (PISA_BF16) or stats->H (PISA_FP32) non-null and
- * written by the pisa_precompute call that wrote the other stats; otherwise PISA_ERR_INVALID_ARG.
- * On the bf16 path it is two launches: the attention kernel, which also leaves each row's softmax
- * offset and 1/D_t in ws, then a tensor-core kernel that adds s sum_j alpha_{t,j} q_t (H_j - Hbar)
- * / D_t to o over the unselected blocks (o is read back in bf16 and rounded once more). */
+ * written by the pisa_precompute call that wrote the other stats, and on the bf16 path ws_bytes >=
+ * pisa_perblock_workspace_bytes(shape); otherwise PISA_ERR_INVALID_ARG.  On the bf16 path it is
+ * two launches: the attention kernel, which leaves its fp32 output and each row's softmax offset
+ * and 1/D_t in ws, then a tensor-core kernel that adds s sum_j alpha_{t,j} q_t (H_j - Hbar) / D_t
+ * over the unselected blocks and writes o.  With keep_k == nb it is the PISA_MODE_PISA call. */
 PISA_API pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k, const void* v,
                            const pisa_stats* stats, const int32_t* sel, const int32_t* order,
                            int32_t keep_k, int32_t mode, void* o, void* ws, size_t ws_bytes,

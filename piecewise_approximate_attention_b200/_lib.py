@@ -20,7 +20,7 @@ PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
            "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string",
-           "pisa_precompute_noalloc", "pisa_testing_set_attention_fault")
+           "pisa_precompute_noalloc", "pisa_testing_set_attention_fault", "pisa_perblock_workspace_bytes")
 
 
 class PisaShape(ctypes.Structure):
@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
             "pisa_stats_bytes": (sz, [P(PisaShape), i32]),
             "pisa_stats_carve": (i32, [P(PisaShape), vp, sz, i32, P(PisaStats)]),
             "pisa_workspace_bytes": (sz, [P(PisaShape)]),
+            "pisa_perblock_workspace_bytes": (sz, [P(PisaShape)]),
             "pisa_precompute": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, sz, vp]),
             "pisa_route": (i32, [P(PisaShape), P(PisaStats), i32, f32, vp, vp, vp, vp]),
             "pisa_attention": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, vp, i32, i32, vp, vp, sz, vp]),
@@ -173,9 +174,16 @@ def alloc_stats(shape: PisaShape, device, with_H: bool = False) -> Stats:
                  view(st.hdiff_op, bf, (B, H, nb, d, d)))
 
 
-def alloc_workspace(shape: PisaShape, device):
+def pisa_perblock_workspace_bytes(shape: PisaShape) -> int:
+    return int(lib().pisa_perblock_workspace_bytes(ctypes.byref(shape)))
+
+
+def alloc_workspace(shape: PisaShape, device, per_block: bool = False):
+    """Zeroed device workspace (the status word must start at zero); per_block sizes it for
+    PISA_MODE_PER_BLOCK."""
     import torch
-    return torch.zeros(pisa_workspace_bytes(shape), dtype=torch.uint8, device=device)
+    n = pisa_perblock_workspace_bytes(shape) if per_block else pisa_workspace_bytes(shape)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def pisa_precompute(shape: PisaShape, q, k, v, stats: Stats, ws, stream=None):

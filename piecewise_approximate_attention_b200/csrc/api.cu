@@ -142,6 +142,14 @@ size_t pisa_workspace_bytes(const pisa_shape* shape) {
   return kStatusBytes + (pre > rows ? pre : rows);
 }
 
+size_t pisa_perblock_workspace_bytes(const pisa_shape* shape) {
+  Dims g;
+  if (check_shape(shape, &g) != PISA_OK) return 0;
+  const size_t base = pisa_workspace_bytes(shape);
+  const size_t pb = perblock_ws_bytes(g);
+  return pb > base ? pb : base;
+}
+
 pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
                             const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream) {
   Dims g;
@@ -186,6 +194,8 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
   if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
   if (mode == PISA_MODE_PER_BLOCK && !(g.dtype == PISA_BF16 ? stats->hdiff_op : stats->H)) return PISA_ERR_INVALID_ARG;
   if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
+  const bool per_block = mode == PISA_MODE_PER_BLOCK && keep_k < g.nb;
+  if (per_block && g.dtype == PISA_BF16 && ws_bytes < pisa_perblock_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   int* status = static_cast<int*>(ws);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (g.dtype == PISA_BF16) {
@@ -198,16 +208,18 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
         !encode_bf16_3d(&maps.hbar, stats->hbar_op, g.d, g.d, bh, 128))
       return PISA_ERR_CUDA;
     const unsigned long long wait_ns = g_test_wait_ns ? g_test_wait_ns : kWaitLimitNs;
-    // per-block mode: the attention kernel runs in PISA mode and leaves each row's softmax offset and
-    // 1/D_t behind; the second kernel adds the per-block minus global first-order difference
-    const bool per_block = mode == PISA_MODE_PER_BLOCK && keep_k < g.nb;
-    float2* rows = per_block ? reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes) : nullptr;
+    // per-block mode: the attention kernel runs in PISA mode, leaves each row's softmax offset and
+    // 1/D_t and its fp32 output in ws; the second kernel adds the per-block minus global first-order
+    // difference and writes o (one rounding to bf16)
+    char* wsb = static_cast<char*>(ws);
+    float2* rows = per_block ? reinterpret_cast<float2*>(wsb + kStatusBytes) : nullptr;
+    float* o32 = per_block ? reinterpret_cast<float*>(wsb + o32_offset(g)) : nullptr;
     cudaError_t e = launch_attention_sm100(g, maps, sel, order, keep_k, mode == PISA_MODE_EXACT_ONLY ? mode : PISA_MODE_PISA,
-                                           stats->vscale, o, rows, status, wait_ns, g_test_fault, cs);
+                                           stats->vscale, o, rows, o32, status, wait_ns, g_test_fault, cs);
     if (e != cudaSuccess || !per_block) return cuda_status(e);
     CUtensorMap hmap;
     if (!encode_bf16_3d(&hmap, stats->hdiff_op, g.d, (uint64_t)g.nb * g.d, bh, 128)) return PISA_ERR_CUDA;
-    return cuda_status(launch_perblock_sm100(g, maps, hmap, sel, order, keep_k, rows, o, status, wait_ns, cs));
+    return cuda_status(launch_perblock_sm100(g, maps, hmap, sel, order, keep_k, rows, o32, o, status, wait_ns, cs));
   }
   return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status, cs));
 }

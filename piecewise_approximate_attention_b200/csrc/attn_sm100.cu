@@ -78,6 +78,7 @@ struct Params {
   const int32_t* order;
   __nv_bfloat16* o;
   float2* rowstats;          // nullable [B*H][L]: (softmax offset m*s*log2(e), 1/D_t) per row
+  float* o32;                // nullable [B*H][L][D]: the output in fp32 instead of bf16 in o
   int* status;
   unsigned long long wait_ns;
 };
@@ -524,10 +525,24 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           }
           pk[x >> 1] = pack_bf16x2(a * inv, b * inv);
         }
-        if (row_valid) {
+        if (row_valid && !p.o32) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * ch);
 #pragma unroll
           for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        }
+        if (row_valid && p.o32) {
+          float4* dst = reinterpret_cast<float4*>(p.o32 + grow_idx * D + 32 * ch);
+#pragma unroll
+          for (int x = 0; x < 32; x += 4) {
+            float a0 = ov[x] * vsc, a1 = ov[x + 1] * vsc, a2 = ov[x + 2] * vsc, a3 = ov[x + 3] * vsc;
+            if (need_corr) {
+              a0 = fmaf(A, cv[x], a0);
+              a1 = fmaf(A, cv[x + 1], a1);
+              a2 = fmaf(A, cv[x + 2], a2);
+              a3 = fmaf(A, cv[x + 3], a3);
+            }
+            dst[x >> 2] = make_float4(a0 * inv, a1 * inv, a2 * inv, a3 * inv);
+          }
         }
       }
     }
@@ -545,7 +560,8 @@ size_t attention_sm100_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
                                    int keep_k, int mode, const float* vscale, void* o, float2* rowstats,
-                                   int* status, unsigned long long wait_ns, int fault, cudaStream_t stream) {
+                                   float* o32, int* status, unsigned long long wait_ns, int fault,
+                                   cudaStream_t stream) {
   Params p;
   p.L = g.L;
   p.nb = g.nb;
@@ -561,6 +577,7 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
   p.order = order;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.rowstats = rowstats;
+  p.o32 = o32;
   p.status = status;
   p.wait_ns = wait_ns;
   const size_t smem = attention_sm100_smem_bytes();

@@ -29,8 +29,11 @@ inline size_t partials_bytes(const Dims& g) {
 // after the partials: per (head, group of blocks) max |v|, which sets the head's value scale
 inline size_t vmax_bytes(const Dims& g) { return (size_t)g.BH() * num_parts(g) * sizeof(float); }
 inline size_t vmax_offset(const Dims& g) { return kStatusBytes + ((partials_bytes(g) + 255) / 256) * 256; }
-// per-block first-order mode: per query row (softmax offset in log2 units, 1 / D_t), at kStatusBytes
+// per-block first-order mode: per query row (softmax offset in log2 units, 1 / D_t) at kStatusBytes,
+// then the attention output in fp32 (rounded to bf16 once, after the per-block term is added)
 inline size_t rowstats_bytes(const Dims& g) { return (size_t)g.BH() * g.L * 2 * sizeof(float); }
+inline size_t o32_offset(const Dims& g) { return kStatusBytes + (rowstats_bytes(g) + 255) / 256 * 256; }
+inline size_t perblock_ws_bytes(const Dims& g) { return o32_offset(g) + (size_t)g.BH() * g.L * g.d * sizeof(float); }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -77,10 +80,12 @@ cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float 
                          int32_t* order, float* scores, cudaStream_t stream);
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
                                    int keep_k, int mode, const float* vscale, void* o, float2* rowstats,
-                                   int* status, unsigned long long wait_ns, int fault, cudaStream_t stream);
+                                   float* o32, int* status, unsigned long long wait_ns, int fault,
+                                   cudaStream_t stream);
 cudaError_t launch_perblock_sm100(const Dims& g, const AttnMaps& maps, const CUtensorMap& hdiff,
                                   const int32_t* sel, const int32_t* order, int keep_k, const float2* rowstats,
-                                  void* o, int* status, unsigned long long wait_ns, cudaStream_t stream);
+                                  const float* o32, void* o, int* status, unsigned long long wait_ns,
+                                  cudaStream_t stream);
 cudaError_t launch_attention_simt(const Dims& g, const void* q, const void* k, const void* v,
                                   const pisa_stats& st, const int32_t* sel, int keep_k, int mode,
                                   void* o, int* status, cudaStream_t stream);

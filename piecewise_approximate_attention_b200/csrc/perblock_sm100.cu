@@ -3,10 +3,10 @@
 // "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion Transformers", §2 핵심 알고리즘:
 // the first-order term of an unselected block j is s (q_t H_j) alpha_tj; the method replaces every
 // H_j by their mean Hbar so that no block's d x d matrix has to be loaded.  This kernel measures
-// what that costs: after the attention kernel (global Hbar) has written o_t and left each row's
-// softmax offset and 1/D_t behind, it adds
-//     o_t += s sum_{j in U_i} alpha_tj q_t (H_j - Hbar) / D_t,     alpha_tj = exp(s q_t.kbar_j - offset_t)
-// so that o_t becomes the per-block first-order result.
+// what that costs: after the attention kernel (global Hbar) has left its output o_t in fp32 and each
+// row's softmax offset and 1/D_t in the workspace, it writes
+//     o_t = bf16( o_t + s sum_{j in U_i} alpha_tj q_t (H_j - Hbar) / D_t ),   alpha_tj = exp(s q_t.kbar_j - offset_t)
+// the per-block first-order result, rounded to bf16 once.
 //
 // Mapping onto B200 (one CTA = one 128-row query tile, the same tiles and query-block pairs as the
 // attention kernel; one CTA per SM, 512 TMEM columns):
@@ -14,12 +14,12 @@
 //   * For each block j that the tile's query blocks did not both select, the four row warps build
 //     W_j = alpha_tj q_t (one row per thread, bf16, q_t held in registers) in TMEM, and the MMA warp
 //     accumulates O += W_j (s (H_j - Hbar)), A = W_j from TMEM, B = the block's 128 x 128 bf16
-//     matrix streamed by TMA through a three-stage ring.  W has two TMEM slots, so building W_{j+1}
-//     overlaps the MMAs of W_j.  Rows whose own query block selected j get alpha = 0.
-//   * The epilogue reads O from TMEM and adds it to the bf16 output row.
+//     matrix streamed by TMA through a ring of shared-memory stages.  W has several TMEM slots, so
+//     building the next W overlaps the MMAs of the current one.  Rows whose own query block selected j get alpha = 0.
+//   * The epilogue reads O from TMEM, adds the row's fp32 attention output and writes bf16.
 // Warp roles: warps 0-3 W builders + epilogue (TMEM lanes 0-127), warp 4 TMA producer, warp 5 MMA
 // issuer and TMEM owner.  Every mbarrier wait is bounded; on a timeout the CTA sets the status
-// word, drains its own copies and MMAs, frees TMEM and leaves o unchanged for its rows.
+// word, drains its own copies and MMAs, frees TMEM and leaves its rows of o unwritten.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -33,9 +33,17 @@ constexpr int D = 128;
 constexpr int kThreads = 192;
 constexpr int kHalf = 128 * 64 * 2;        // 128 rows x 64 bf16 columns, 128B-swizzled: 16 KB
 constexpr int kTileBytes = 2 * kHalf;
-constexpr int kHS = 3;                     // stages of the per-block matrix ring
+#ifndef PISA_PB_HSTAGES
+#define PISA_PB_HSTAGES 3
+#endif
+#ifndef PISA_PB_WSLOTS
+#define PISA_PB_WSLOTS 2
+#endif
+constexpr int kHS = PISA_PB_HSTAGES;       // stages of the per-block matrix ring
+constexpr int kWS = PISA_PB_WSLOTS;        // W buffers in TMEM
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColC = 0, kColW = 128, kColO = 256;   // C: 128 cols, W: 2 x 64 cols, O: 128 cols
+constexpr uint32_t kColC = 0, kColW = 128, kColO = 128 + 64 * kWS;   // C: 128 cols, W: kWS x 64, O: 128
+static_assert(kColO + 128 <= kTmemCols, "TMEM columns");
 constexpr int kWords = 128;                // selection bitmap words (nb <= 4096)
 constexpr int kAlphaStride = 33;
 
@@ -45,7 +53,7 @@ struct alignas(1024) Smem {
   uint8_t h[kHS][kTileBytes];
   float alpha[128 * kAlphaStride];          // alpha of the current 32 centroids, one row per thread
   uint64_t bar_q, bar_kfull, bar_kempty, bar_cfull, bar_cempty;
-  uint64_t bar_hfull[kHS], bar_hempty[kHS], bar_wfull[2], bar_wempty[2];
+  uint64_t bar_hfull[kHS], bar_hempty[kHS], bar_wfull[kWS], bar_wempty[kWS];
   uint64_t bar_final, bar_drain;
   uint32_t tmem_base;
   int abort;
@@ -60,6 +68,7 @@ struct Params {
   const int32_t* sel;
   const int32_t* order;
   const float2* rowstats;
+  const float* o32;          // [B*H][L][D] attention output with the global first-order term, fp32
   __nv_bfloat16* o;
   int* status;
   unsigned long long wait_ns;
@@ -77,6 +86,20 @@ __device__ __forceinline__ uint32_t proc_word(const Smem& sm, int w, int nb) {
   const int r = nb - 32 * w;
   const uint32_t valid = r >= 32 ? 0xffffffffu : (r > 0 ? ((1u << r) - 1u) : 0u);
   return valid & ~(sm.bitsA[w] & sm.bitsB[w]);
+}
+
+// o row = bf16(o32 row + add[0..127]) for the 32 columns starting at 32*ch
+__device__ __forceinline__ void store_row32(const Params& p, size_t row, int ch, const float* add) {
+  const float4* src = reinterpret_cast<const float4*>(p.o32 + row * D + 32 * ch);
+  uint4* dst = reinterpret_cast<uint4*>(p.o + row * D + 32 * ch);
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const float4 a = src[2 * x], b = src[2 * x + 1];
+    dst[x] = make_uint4(pack_bf16x2(a.x + add[8 * x], a.y + add[8 * x + 1]),
+                        pack_bf16x2(a.z + add[8 * x + 2], a.w + add[8 * x + 3]),
+                        pack_bf16x2(b.x + add[8 * x + 4], b.y + add[8 * x + 5]),
+                        pack_bf16x2(b.z + add[8 * x + 6], b.w + add[8 * x + 7]));
+  }
 }
 
 __device__ __forceinline__ bool wait_or_abort(Smem& sm, uint64_t* bar, uint32_t parity, const Params& p) {
@@ -140,7 +163,7 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
       mbar_init(&sm.bar_hfull[i], 1);
       mbar_init(&sm.bar_hempty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kWS; ++i) {
       mbar_init(&sm.bar_wfull[i], 128);
       mbar_init(&sm.bar_wempty[i], 1);
     }
@@ -150,7 +173,19 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
     fence_mbar_init();
   }
   __syncthreads();
-  if (sm.nproc == 0) return;      // every block of this tile was attended exactly: nothing to add
+  if (sm.nproc == 0) {
+    // every block of this tile was attended exactly: nothing to add, only the rounding to bf16
+    if (threadIdx.x < 128) {
+      const int r = threadIdx.x;
+      const bool upper = pair && r >= 64;
+      const int myq = upper ? qb : qa, rloc = pair ? (r & 63) : r;
+      if (rloc < block_count(myq, p.L, p.block) && (!upper || has_b)) {
+        const float zero[32] = {};
+        for (int ch = 0; ch < 4; ++ch) store_row32(p, (size_t)bh * p.L + (size_t)myq * p.block + rloc, ch, zero);
+      }
+    }
+    return;
+  }
   if (warp == 5) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -226,8 +261,8 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
         mma_commit(&sm.bar_cfull);
         for (int w = 4 * ct; w < 4 * ct + 4 && ok; ++w) {
           for (uint32_t pm = proc_word(sm, w, p.nb); pm; pm &= pm - 1) {
-            const int slot = n & 1, s = n % kHS;
-            if (!(ok = wait_or_abort(sm, &sm.bar_wfull[slot], (n >> 1) & 1, p))) break;
+            const int slot = n % kWS, s = n % kHS;
+            if (!(ok = wait_or_abort(sm, &sm.bar_wfull[slot], (n / kWS) & 1, p))) break;
             if (!(ok = wait_or_abort(sm, &sm.bar_hfull[s], (n / kHS) & 1, p))) break;
             tc_fence_after();
             const uint64_t hd = smem_desc_sw128(smem_u32(sm.h[s]), kHalf, 1024);
@@ -293,9 +328,9 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
         for (int x = 0; x < 32; ++x)
           arow[x] = ((am >> x) & 1u) ? ex2(fmaf(c[x], p.scale_log2, -rs.x)) * rs.y : 0.f;
         for (uint32_t mm = pm; mm; mm &= mm - 1) {
-          const int x = __ffs(mm) - 1, slot = n & 1;
-          if (n >= 2) {
-            ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_wempty[slot], ((n >> 1) - 1) & 1, p));
+          const int x = __ffs(mm) - 1, slot = n % kWS;
+          if (n >= kWS) {
+            ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_wempty[slot], ((n / kWS) - 1) & 1, p));
             if (!ok) break;
             tc_fence_after();
           }
@@ -319,28 +354,12 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
     if (ok) ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_final, 0, p));
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* orow = p.o + grow_idx * D;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float ov[32];
         tmem_ld32(trow + kColO + 32 * ch, ov);
         tmem_ld_wait();
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * ch);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const uint4 u = dst[x];
-            const uint32_t in[4] = {u.x, u.y, u.z, u.w};
-            uint32_t out[4];
-#pragma unroll
-            for (int y = 0; y < 4; ++y) {
-              const float lo = __uint_as_float(in[y] << 16) + ov[8 * x + 2 * y];
-              const float hi = __uint_as_float(in[y] & 0xffff0000u) + ov[8 * x + 2 * y + 1];
-              out[y] = pack_bf16x2(lo, hi);
-            }
-            dst[x] = make_uint4(out[0], out[1], out[2], out[3]);
-          }
-        }
+        if (row_valid) store_row32(p, grow_idx, ch, ov);
       }
     }
   }
@@ -355,7 +374,8 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
 
 cudaError_t launch_perblock_sm100(const Dims& g, const AttnMaps& maps, const CUtensorMap& hdiff,
                                   const int32_t* sel, const int32_t* order, int keep_k, const float2* rowstats,
-                                  void* o, int* status, unsigned long long wait_ns, cudaStream_t stream) {
+                                  const float* o32, void* o, int* status, unsigned long long wait_ns,
+                                  cudaStream_t stream) {
   Params p;
   p.L = g.L;
   p.nb = g.nb;
@@ -365,6 +385,7 @@ cudaError_t launch_perblock_sm100(const Dims& g, const AttnMaps& maps, const CUt
   p.sel = sel;
   p.order = order;
   p.rowstats = rowstats;
+  p.o32 = o32;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.status = status;
   p.wait_ns = wait_ns;

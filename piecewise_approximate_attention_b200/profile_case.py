@@ -1,6 +1,7 @@
 """Runs the PISA hot path a few times on one workload, for profilers (ncu) to capture.
 
     python -m piecewise_approximate_attention_b200.profile_case --workload video-dit-large --heads 8 --iters 3
+    python -m piecewise_approximate_attention_b200.profile_case --heads 4 --iters 2 --mode per_block
 """
 from __future__ import annotations
 
@@ -10,6 +11,7 @@ import argparse
 def main():
     import torch
 
+    from . import _lib as C
     from .runtime import Pisa
     from .workloads import WORKLOADS, make_qkv
 
@@ -17,17 +19,19 @@ def main():
     ap.add_argument("--workload", default="video-dit-large")
     ap.add_argument("--heads", type=int, default=8)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--mode", choices=("pisa", "per_block"), default="pisa")
     a = ap.parse_args()
+    mode = C.PISA_MODE_PER_BLOCK if a.mode == "per_block" else C.PISA_MODE_PISA
     w = WORKLOADS[a.workload].with_(heads=a.heads)
     q, k, v = (x.cuda() for x in make_qkv(w))
     B, H, L, d = q.shape
-    p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, "cuda")
+    p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, "cuda", mode)
     o = torch.empty_like(q)
     for _ in range(a.iters):
         p(q, k, v, o)
     torch.cuda.synchronize()
     st = p.device_error()
-    print(f"{w.name} heads={H} L={L} block={w.block} keep_k={w.keep_k} iters={a.iters} status={st}")
+    print(f"{w.name} heads={H} L={L} block={w.block} keep_k={w.keep_k} mode={a.mode} iters={a.iters} status={st}")
     if st[0] != 0:
         raise SystemExit(1)
 

@@ -30,7 +30,7 @@ class Pisa:
         if mode == C.PISA_MODE_PER_BLOCK:
             with_H = True         # the per-block first-order matrices live in the stats
         self.stats = C.alloc_stats(self.shape, self.device, with_H)
-        self.ws = C.alloc_workspace(self.shape, self.device)
+        self.ws = C.alloc_workspace(self.shape, self.device, per_block=mode == C.PISA_MODE_PER_BLOCK)
         self.sel = torch.empty((batch, heads, self.nb, max(keep_k, 1)), dtype=torch.int32, device=self.device)
         self.order = torch.empty((batch, heads, self.nb), dtype=torch.int32, device=self.device) if pair else None
 

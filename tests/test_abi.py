@@ -63,6 +63,9 @@ def test_stats_bytes_and_carve_are_host_only():
     assert C.lib().pisa_stats_carve(ctypes.byref(sh), base + 16, n1, 1, ctypes.byref(st)) == C.PISA_ERR_INVALID_ARG
     assert C.lib().pisa_stats_carve(ctypes.byref(sh), base, n1 - 1, 1, ctypes.byref(st)) == C.PISA_ERR_INVALID_ARG
     assert C.pisa_workspace_bytes(sh) >= 256 + 2 * 1 * 128 * 128 * 4
+    # per-block mode: status word, per-row offsets and 1/D_t, the fp32 output
+    assert C.pisa_perblock_workspace_bytes(sh) >= 256 + 2 * 1000 * 8 + 2 * 1000 * 128 * 4
+    assert C.pisa_perblock_workspace_bytes(sh) >= C.pisa_workspace_bytes(sh)
     # fp32 mode needs no tensor-core operand copies
     f32 = _shape(dtype="fp32")
     st32 = C.PisaStats()
@@ -95,6 +98,7 @@ def test_bad_shapes_rejected(kw, expect):
     assert C.lib().pisa_precompute(ctypes.byref(sh), 16, 16, 16, ctypes.byref(st), 16, 1 << 30, None) == expect
     assert C.pisa_stats_bytes(sh, False) == 0
     assert C.pisa_workspace_bytes(sh) == 0
+    assert C.pisa_perblock_workspace_bytes(sh) == 0
 
 
 def _fake_stats(sh):
@@ -130,8 +134,15 @@ def test_invalid_arguments_rejected_without_launch():
                                                                   mode, o, P, wsb, None)
     assert att(4, 3) == C.PISA_ERR_INVALID_ARG
     assert att(4, -1) == C.PISA_ERR_INVALID_ARG
-    # the per-block first-order mode needs the per-block operand copy in the stats
+    # the per-block first-order mode needs the per-block operand copy in the stats and the larger
+    # workspace
     assert att(4, C.PISA_MODE_PER_BLOCK) == C.PISA_ERR_INVALID_ARG
+    sth = C.PisaStats()
+    nh = C.pisa_stats_bytes(sh, True)
+    assert L.pisa_stats_carve(bs, 1 << 24, nh, 1, ctypes.byref(sth)) == C.PISA_OK
+    assert sth.hdiff_op
+    assert L.pisa_attention(bs, P, P, P, ctypes.byref(sth), P, None, 4, C.PISA_MODE_PER_BLOCK, P, P, ws,
+                            None) == C.PISA_ERR_INVALID_ARG
     assert att(0, C.PISA_MODE_EXACT_ONLY) == C.PISA_ERR_INVALID_ARG
     assert att(17, C.PISA_MODE_PISA) == C.PISA_ERR_INVALID_ARG
     assert att(4, C.PISA_MODE_PISA, sel=None) == C.PISA_ERR_INVALID_ARG

@@ -296,8 +296,9 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           ++issued_k;
         }
       }
-      if (!ok) {
-        // drain: every copy issued so far must land before this CTA's shared memory is released
+      {
+        // drain: every copy issued must land before this CTA's shared memory is released (in a
+        // normal run the MMA warp has waited for all of them, so these waits return at once)
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
         for (int i = max(0, issued_k - kKS); i < issued_k; ++i)

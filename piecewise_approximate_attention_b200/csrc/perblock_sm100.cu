@@ -230,7 +230,9 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
           }
         }
       }
-      if (!ok) {
+      {
+        // every copy issued must land before this CTA's shared memory is released (normally the
+        // MMA warp has already waited for all of them)
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
         if (issued_k > 0)

@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
         tma_load_3d(sm.v[s] + kHalf, &maps.v, &sm.full[s], 64, y, bh);
         ++issued;
       }
-      if (!ok) {   // let issued copies land before shared memory is released
+      {   // let issued copies land before shared memory is released (normally already landed)
         const uint64_t t0 = globaltimer_ns();
         for (int t = max(0, issued - 2); t < issued; ++t)
           while (!mbar_try_wait(&sm.full[t & 1], (t >> 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
         tma_load_3d(sm.v[s] + kHalf, &maps.v, &sm.full[s], 64, y, bh);
         ++issued;
       }
-      if (!ok) {
+      {   // let issued copies land before shared memory is released (normally already landed)
         const uint64_t t0 = globaltimer_ns();
         for (int t = max(0, issued - kStagesB); t < issued; ++t)
           while (!mbar_try_wait(&sm.full[t % kStagesB], (t / kStagesB) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}

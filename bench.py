@@ -226,6 +226,7 @@ def run_ours(args, rank, world, local_rank):
     per_block = per_block_variant(p, w, (qd, kd, vd), o_dense, stream, time_calls)
     per_block["rel_l2_vs_dense"]["keep_or_drop"] = round(rel_keep_or_drop, 6)
     del o_dense
+    short = short_sequences(dev) if not args.no_extras else None
 
     # end to end through the public API with host buffers: H2D of q, k, v and D2H of o every step
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
@@ -296,6 +297,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": args.steps * p.launches_per_step(),
         "clocks": clk,
         "per_block_first_order": per_block,
+        "short_sequences": short,
     }
     if rank == 0:
         result["cpu_baseline"] = cpu_baseline(w)
@@ -354,6 +356,56 @@ def per_block_variant(p, w, qkv, o_dense, stream, time_calls):
     return out
 
 
+SHORT_WORKLOADS = ("image-dit", "sweep-L8192-s0.875")
+
+
+def short_sequences(dev, steps: int = 20):
+    """Short sequences, where per-launch overhead and the pre-computation weigh most: the full
+    step (pre-compute + route + attention) launched call by call and replayed as one CUDA graph,
+    its parts, and the library's dense attention on the same inputs.  Outside the timed region."""
+    import torch
+    from piecewise_approximate_attention_b200.runtime import Pisa
+    from piecewise_approximate_attention_b200.workloads import WORKLOADS, make_qkv
+    out = {}
+    for name in SHORT_WORKLOADS:
+        w = WORKLOADS[name]
+        q, k, v = (x.to(dev) for x in make_qkv(w))
+        B, H, L, d = q.shape
+        p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, dev)
+        o = torch.empty_like(q)
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+
+        def timed(fn):
+            for _ in range(3):
+                fn()
+            a, b = ev(), ev()
+            torch.cuda.synchronize()
+            a.record()
+            for _ in range(steps):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / steps
+
+        direct = timed(lambda: p(q, k, v, o))
+        pre = timed(lambda: p.precompute(q, k, v))
+        route = timed(lambda: p.route())
+        attn = timed(lambda: p.attention(q, k, v, o))
+        graph = p.capture(q, k, v, o)
+        replay = timed(graph.replay)
+        dense = Pisa(B, H, L, d, w.block, p.nb, w.lam, w.dtype, 1.0, dev, pair=False)
+        dense.precompute(q, k, v)
+        dense.route()
+        dense_ms = timed(lambda: dense.attention(q, k, v, o))
+        out[name] = {"seq_len": L, "heads": H, "keep_k": w.keep_k, "num_blocks": p.nb,
+                     "ms_step_launches": round(direct, 4), "ms_step_graph": round(replay, 4),
+                     "ms_precompute": round(pre, 4), "ms_route": round(route, 4), "ms_attention": round(attn, 4),
+                     "ms_dense_attention": round(dense_ms, 4),
+                     "speedup_step_vs_dense": round(dense_ms / replay, 3)}
+        del graph, p, dense
+    return out
+
+
 def cpu_baseline(w, heads=(0,)):
     """fp64 oracle on a bounded sample (one full head of the workload) on the host cores."""
     import numpy as np
@@ -405,6 +457,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-extras", action="store_true", help="skip the short-sequence measurements")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

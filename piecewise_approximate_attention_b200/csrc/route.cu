@@ -228,19 +228,16 @@ __global__ void __launch_bounds__(kThreads) pair_kernel(const int32_t* __restric
       for (int a = 0; a < kChunk && c0 + a < nb; ++a) {
         const int i = c0 + a;
         if ((used[i >> 5] >> (i & 31)) & 1u) continue;
-        int best = -1, bestv = -1;
+        // best partner: most shared key blocks, ties to the nearer one; packed as
+        // ((overlap + 1) << 8) | (255 - distance) so one warp max reduction picks it (0 = none)
+        uint32_t key = 0u;
         for (int dl = lane + 1; dl <= kWin; dl += 32) {
           const int p = i + dl;
-          if (p < nb && !((used[p >> 5] >> (p & 31)) & 1u)) {
-            const int val = ov[a * kWin + dl - 1];
-            if (val > bestv) { bestv = val; best = dl; }
-          }
+          if (p < nb && !((used[p >> 5] >> (p & 31)) & 1u))
+            key = max(key, ((uint32_t)(ov[a * kWin + dl - 1] + 1) << 8) | (uint32_t)(255 - dl));
         }
-        for (int o = 16; o > 0; o >>= 1) {
-          const int ov2 = __shfl_xor_sync(0xffffffffu, bestv, o);
-          const int ob2 = __shfl_xor_sync(0xffffffffu, best, o);
-          if (ov2 > bestv || (ov2 == bestv && ob2 >= 0 && (best < 0 || ob2 < best))) { bestv = ov2; best = ob2; }
-        }
+        key = __reduce_max_sync(0xffffffffu, key);
+        const int best = key ? 255 - (int)(key & 255u) : -1;
         if (lane == 0) {
           used[i >> 5] |= 1u << (i & 31);
           if (best > 0) {

@@ -55,6 +55,24 @@ class Pisa:
         self.attention(q, k, v, o, stream=stream)
         return o
 
+    def capture(self, q, k, v, o):
+        """Records one full step (pre-computation, routing, attention of q, k, v into o) as a CUDA
+        graph and returns it; ``graph.replay()`` then re-runs the step on whatever the same
+        buffers hold, with one launch from the host.  The buffers must stay allocated while the
+        graph is used.  The step runs once eagerly first (outside the capture)."""
+        import torch
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            self(q, k, v, o)
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self.precompute(q, k, v)
+            self.route()
+            self.attention(q, k, v, o)
+        return graph
+
     def launches_per_step(self) -> int:
         """Kernels one __call__ enqueues: pre-compute 3, routing 1 (+1 pairing), attention 1 (+1 for
         the per-block first-order kernel on the bf16 path)."""

@@ -232,3 +232,30 @@ def test_bad_selection_is_reported_not_faulted():
     torch.cuda.synchronize()
     assert p.device_error() == (C.PISA_ERR_INVALID_ARG, C.PISA_DEVERR_BAD_SELECTION)
     assert p.device_error() == (C.PISA_OK, 0)
+
+
+def test_graph_replay_matches_direct_calls():
+    """A captured step (pre-compute, route, attention) replays to the same output as direct calls,
+    and follows new inputs written into the captured buffers."""
+    w = WORKLOADS["image-dit"].with_(heads=4)
+    q, k, v = (x.cuda() for x in make_qkv(w))
+    B, H, L, d = q.shape
+    p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, "cuda")
+    o_direct = torch.empty_like(q)
+    p(q, k, v, o_direct)
+    o = torch.empty_like(q)
+    g = p.capture(q, k, v, o)
+    o.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_direct)
+    q2, k2, v2 = (x.cuda() for x in make_qkv(w, seed=9))
+    q.copy_(q2)
+    k.copy_(k2)
+    v.copy_(v2)
+    g.replay()
+    o2 = torch.empty_like(q)
+    p(q2, k2, v2, o2)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2)
+    assert p.device_error() == (C.PISA_OK, 0)

@@ -225,6 +225,7 @@ def run_ours(args, rank, world, local_rank):
     del dense
     per_block = per_block_variant(p, w, (qd, kd, vd), o_dense, stream, time_calls)
     per_block["rel_l2_vs_dense"]["keep_or_drop"] = round(rel_keep_or_drop, 6)
+    reordering = token_reordering(p, w, (qd, kd, vd), o_dense, stream, time_calls) if not args.no_extras else None
     del o_dense
     short = short_sequences(dev) if not args.no_extras else None
 
@@ -298,6 +299,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "per_block_first_order": per_block,
         "short_sequences": short,
+        "token_reordering": reordering,
     }
     if rank == 0:
         result["cpu_baseline"] = cpu_baseline(w)
@@ -354,6 +356,58 @@ def per_block_variant(p, w, qkv, o_dense, stream, time_calls):
     }
     del pb
     return out
+
+
+def token_reordering(p, w, qkv, o_dense, stream, time_calls):
+    """PARO-style token reordering on the bench workload, outside the timed region: the gather
+    kernel's bandwidth (one [B,H,L,d] tensor in, one out) and PISA's distance to dense attention
+    when its blocks follow each axis order of the frames x height x width grid, and with the order
+    chosen per head by the smallest sum_j M_j."""
+    import torch
+    from piecewise_approximate_attention_b200.runtime import (AXIS_ORDERS, axis_order_permutations,
+                                                             choose_axis_order, reorder_tokens, restore_tokens)
+    qd, kd, vd = qkv
+    perms = axis_order_permutations(w.grid, w.text_tokens, qd.device)
+    buf = [torch.empty_like(qd) for _ in range(3)]
+    o_r = torch.empty_like(qd)
+    o = torch.empty_like(qd)
+    gather_ms = time_calls(lambda: reorder_tokens(qd, perms[3], out=buf[0], stream=stream))
+    moved = 2 * qd.numel() * qd.element_size()
+    _, _, hbm, _ = _peaks()
+    out = {"gather_ms_per_tensor": round(gather_ms, 4), "gather_gbs": round(moved / (gather_ms * 1e-3) / 1e9, 1),
+           "gather_frac_of_hbm": round(moved / (gather_ms * 1e-3) / 1e9 / hbm, 4), "rel_l2_vs_dense": {}}
+
+    def run(perm):
+        for x, b in zip(qkv, buf):
+            reorder_tokens(x, perm, out=b, stream=stream)
+        p.precompute(*buf, stream=stream)
+        p.route(stream=stream)
+        p.attention(*buf, o_r, stream=stream)
+        restore_tokens(o_r, perm, out=o, stream=stream)
+        torch.cuda.synchronize()
+        return rel_l2(o, o_dense)
+
+    for r, order in enumerate(AXIS_ORDERS):
+        out["rel_l2_vs_dense"][order] = round(run(perms[r]), 6)
+    with torch.cuda.stream(stream):
+        chosen, idx = choose_axis_order(p, qd, kd, vd, perms)
+    out["rel_l2_vs_dense"]["per_head_min_spread"] = round(run(chosen), 6)
+    out["per_head_order_counts"] = {o: int((idx == r).sum()) for r, o in enumerate(AXIS_ORDERS)}
+    step_ms = time_calls(lambda: run_step_reordered(p, qkv, buf, o_r, o, chosen, stream))
+    out["ms_step_with_reordering"] = round(step_ms, 4)
+    del buf, o_r, o
+    return out
+
+
+def run_step_reordered(p, qkv, buf, o_r, o, perm, stream):
+    """One step with per-head reordering: gather q, k, v, pre-compute, route, attention, scatter o."""
+    from piecewise_approximate_attention_b200.runtime import reorder_tokens, restore_tokens
+    for x, b in zip(qkv, buf):
+        reorder_tokens(x, perm, out=b, stream=stream)
+    p.precompute(*buf, stream=stream)
+    p.route(stream=stream)
+    p.attention(*buf, o_r, stream=stream)
+    restore_tokens(o_r, perm, out=o, stream=stream)
 
 
 SHORT_WORKLOADS = ("image-dit", "sweep-L8192-s0.875")

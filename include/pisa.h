@@ -179,6 +179,32 @@ PISA_API pisa_status pisa_attention(const pisa_shape* shape, const void* q, cons
                            int32_t keep_k, int32_t mode, void* o, void* ws, size_t ws_bytes,
                            pisa_stream_t stream);
 
+/* Token reordering before blocking ("PAROAttention: Pattern-Aware ReOrdering for Efficient Sparse
+ * and Quantized Attention in Visual Generation Models", abstract: reorder tokens so that attention
+ * patterns become block-wise; the page gives no algorithm, and the reading built here permutes the
+ * axis order of the video's frames x height x width grid, see pisa_axis_permutation).  Copies the
+ * rows of src, a dense [batch_heads, seq_len, row_bytes] tensor, into dst:
+ *   inverse == 0:  dst[h][i] = src[h][perm[i]]     (gather: reorder q, k, v before pisa_precompute)
+ *   inverse != 0:  dst[h][perm[i]] = src[h][i]     (scatter: put the attention output back)
+ * perm: device int32 [seq_len] shared by every head, or [batch_heads, seq_len] when
+ * perm_per_head != 0; it must be a permutation of 0..seq_len-1 (an entry outside that range is
+ * skipped and leaves its row of dst unwritten; a repeated entry leaves the result to write order).
+ * row_bytes: a multiple of 16 (head_dim * element size).  src and dst must not overlap.  Byte copy:
+ * any element type. */
+PISA_API pisa_status pisa_permute_rows(const void* src, void* dst, const int32_t* perm, int32_t batch_heads,
+                                       int32_t seq_len, int32_t row_bytes, int32_t perm_per_head, int32_t inverse,
+                                       pisa_stream_t stream);
+
+/* Host-only helper (perm_host is a HOST buffer of frames*height*width + extra_tokens int32): the
+ * permutation that lists the tokens of a frames x height x width grid, stored in raster order
+ * (t slowest, then h, then w), in the axis order `order` — a NUL-terminated string of the three
+ * distinct characters 't', 'h', 'w', slowest axis first ("thw" is the identity, "hwt" makes the
+ * frame axis the fastest).  perm_host[i] = stored index of the token placed at position i.  The
+ * extra_tokens rows after the grid (e.g. text tokens) keep their place at the end.  Enqueues
+ * nothing; PISA_ERR_INVALID_ARG for a bad order or size. */
+PISA_API pisa_status pisa_axis_permutation(int32_t frames, int32_t height, int32_t width, int32_t extra_tokens,
+                                           const char* order, int32_t* perm_host);
+
 /* Synchronises `stream`, copies the device status word out of ws into *code (0 = clean; otherwise
  * a PISA_DEVERR_* value below) and clears it.  Returns PISA_ERR_DEVICE_TIMEOUT when a bounded wait
  * ran out, PISA_ERR_INVALID_ARG for a bad selection entry, PISA_OK when clean. */

@@ -38,6 +38,7 @@ import numpy as np
 __all__ = [
     "num_blocks", "block_bounds", "block_stats", "route_scores", "route_select",
     "attention_head", "pisa", "dense_attention", "brute_force_head",
+    "axis_permutation", "permute_rows", "pisa_reordered",
 ]
 
 
@@ -316,3 +317,40 @@ def brute_force_head(q, k, v, block: int, sel, scale: float = 1.0, first_order: 
                         Nt[c] += a0 * scale * sum(q[t][a] * Hbar[a][c] for a in range(d))
         out[t] = [x / Dt for x in Nt]
     return out
+
+
+# --------------------------------------------------------------------------------------------
+# Token reordering before blocking
+# ["PAROAttention: Pattern-Aware ReOrdering for Efficient Sparse and Quantized Attention in Visual
+#  Generation Models", abstract: tokens are reordered so that attention becomes block-wise.  The
+#  page gives no algorithm; the reading here permutes the axis order of the frames x height x width
+#  token grid, and the same permutation is applied to q, k and v and undone on the output.]
+# --------------------------------------------------------------------------------------------
+def axis_permutation(grid, order: str, extra_tokens: int = 0) -> np.ndarray:
+    """perm[i] = raster index (t slowest, then h, then w) of the token at position i when the grid
+    is listed with the axes in ``order`` (slowest first); extra tokens keep their place at the end."""
+    T, Hg, W = grid
+    if sorted(order) != ["h", "t", "w"]:
+        raise ValueError(order)
+    raster = np.arange(T * Hg * W).reshape(T, Hg, W)
+    axes = tuple("thw".index(c) for c in order)
+    grid_part = np.transpose(raster, axes).reshape(-1)
+    return np.concatenate([grid_part, np.arange(T * Hg * W, T * Hg * W + extra_tokens)]).astype(np.int64)
+
+
+def permute_rows(x: np.ndarray, perm: np.ndarray, inverse: bool = False) -> np.ndarray:
+    """Gather rows along axis -2 (out[..., i, :] = x[..., perm[i], :]) or, with inverse, scatter
+    them back (out[..., perm[i], :] = x[..., i, :])."""
+    x = np.asarray(x)
+    if not inverse:
+        return x[..., perm, :]
+    out = np.empty_like(x)
+    out[..., perm, :] = x
+    return out
+
+
+def pisa_reordered(q, k, v, perm, block: int, keep_k: int, lam: float, scale: float = 1.0, **kw) -> Dict:
+    """PISA on the reordered sequence, output put back in the original token order."""
+    r = pisa(permute_rows(q, perm), permute_rows(k, perm), permute_rows(v, perm), block, keep_k, lam, scale, **kw)
+    r["o"] = permute_rows(r["o"], perm, inverse=True)
+    return r

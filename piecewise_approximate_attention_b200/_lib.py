@@ -20,7 +20,8 @@ PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
            "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string",
-           "pisa_precompute_noalloc", "pisa_testing_set_attention_fault", "pisa_perblock_workspace_bytes")
+           "pisa_precompute_noalloc", "pisa_testing_set_attention_fault", "pisa_perblock_workspace_bytes",
+           "pisa_permute_rows", "pisa_axis_permutation")
 
 
 class PisaShape(ctypes.Structure):
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
             "pisa_status_string": (ctypes.c_char_p, [i32]),
             "pisa_precompute_noalloc": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp]),
             "pisa_testing_set_attention_fault": (i32, [i32, ctypes.c_uint64]),
+            "pisa_permute_rows": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp]),
+            "pisa_axis_permutation": (i32, [i32, i32, i32, i32, ctypes.c_char_p, P(i32)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -206,6 +209,26 @@ def pisa_attention(shape: PisaShape, q, k, v, stats: Stats, sel, order, keep_k: 
     _check(lib().pisa_attention(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(stats.c), _ptr(sel),
                                 _ptr(order), int(keep_k), int(mode), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)),
            "pisa_attention")
+
+
+def pisa_permute_rows(src, dst, perm, inverse: bool = False, stream=None):
+    """Rows of src [..., L, row] into dst through perm ([L] shared, or one row of perm per head)."""
+    L = src.shape[-2]
+    bh = src.numel() // (L * src.shape[-1])
+    row_bytes = src.shape[-1] * src.element_size()
+    per_head = 1 if perm.dim() > 1 else 0
+    _check(lib().pisa_permute_rows(_ptr(src), _ptr(dst), _ptr(perm), bh, L, row_bytes, per_head, int(bool(inverse)),
+                                   _stream(stream)), "pisa_permute_rows")
+
+
+def pisa_axis_permutation(grid, order: str, extra_tokens: int = 0):
+    """Host int32 numpy permutation of a (frames, height, width) raster grid listed in `order`."""
+    import numpy as np
+    T, Hg, W = grid
+    out = np.empty(T * Hg * W + extra_tokens, dtype=np.int32)
+    _check(lib().pisa_axis_permutation(T, Hg, W, extra_tokens, order.encode(),
+                                       out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))), "pisa_axis_permutation")
+    return out
 
 
 def pisa_read_device_error(ws, stream=None):

@@ -224,6 +224,44 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
   return cuda_status(launch_attention_simt(g, q, k, v, *stats, sel, keep_k, mode, o, status, cs));
 }
 
+pisa_status pisa_permute_rows(const void* src, void* dst, const int32_t* perm, int32_t batch_heads, int32_t seq_len,
+                              int32_t row_bytes, int32_t perm_per_head, int32_t inverse, pisa_stream_t stream) {
+  if (!src || !dst || !perm || !aligned16(src) || !aligned16(dst) || !aligned16(perm)) return PISA_ERR_INVALID_ARG;
+  if (batch_heads < 1 || batch_heads > 65535 || seq_len < 1 || row_bytes < 16 || row_bytes % 16) return PISA_ERR_INVALID_ARG;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(src), b = reinterpret_cast<uintptr_t>(dst);
+  const uintptr_t n = (uintptr_t)batch_heads * (uintptr_t)seq_len * (uintptr_t)row_bytes;
+  if (a < b + n && b < a + n) return PISA_ERR_INVALID_ARG;   // overlapping buffers
+  return cuda_status(launch_permute_rows(src, dst, perm, batch_heads, seq_len, row_bytes, perm_per_head ? 1 : 0,
+                                         inverse ? 1 : 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+pisa_status pisa_axis_permutation(int32_t frames, int32_t height, int32_t width, int32_t extra_tokens,
+                                  const char* order, int32_t* perm_host) {
+  if (frames < 1 || height < 1 || width < 1 || extra_tokens < 0 || !order || !perm_host) return PISA_ERR_INVALID_ARG;
+  if ((long long)frames * height * width + extra_tokens > 0x7fffffffLL) return PISA_ERR_INVALID_ARG;
+  // order: the three axes t, h, w, slowest first
+  int axis[3], seen = 0;
+  for (int i = 0; i < 3; ++i) {
+    const char c = order[i];
+    const int ax = c == 't' ? 0 : c == 'h' ? 1 : c == 'w' ? 2 : -1;
+    if (ax < 0 || (seen >> ax) & 1) return PISA_ERR_INVALID_ARG;
+    seen |= 1 << ax;
+    axis[i] = ax;
+  }
+  if (order[3] != '\0') return PISA_ERR_INVALID_ARG;
+  const int ext[3] = {frames, height, width};
+  // raster (t, h, w) strides of the stored sequence
+  const long long stride[3] = {(long long)height * width, width, 1};
+  const int n0 = ext[axis[0]], n1 = ext[axis[1]], n2 = ext[axis[2]];
+  long long pos = 0;
+  for (int i0 = 0; i0 < n0; ++i0)
+    for (int i1 = 0; i1 < n1; ++i1)
+      for (int i2 = 0; i2 < n2; ++i2)
+        perm_host[pos++] = (int32_t)(i0 * stride[axis[0]] + i1 * stride[axis[1]] + i2 * stride[axis[2]]);
+  for (int e = 0; e < extra_tokens; ++e, ++pos) perm_host[pos] = (int32_t)pos;
+  return PISA_OK;
+}
+
 pisa_status pisa_read_device_error(void* ws, int32_t* code, pisa_stream_t stream) {
   if (!ws || !code || !aligned16(ws)) return PISA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -82,6 +82,8 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
                                    int keep_k, int mode, const float* vscale, void* o, float2* rowstats,
                                    float* o32, int* status, unsigned long long wait_ns, int fault,
                                    cudaStream_t stream);
+cudaError_t launch_permute_rows(const void* src, void* dst, const int32_t* perm, int batch_heads, int L,
+                                int row_bytes, int perm_per_head, int inverse, cudaStream_t stream);
 cudaError_t launch_perblock_sm100(const Dims& g, const AttnMaps& maps, const CUtensorMap& hdiff,
                                   const int32_t* sel, const int32_t* order, int keep_k, const float2* rowstats,
                                   const float* o32, void* o, int* status, unsigned long long wait_ns,

@@ -82,3 +82,44 @@ class Pisa:
 
     def device_error(self, stream=None):
         return C.pisa_read_device_error(self.ws, stream)
+
+
+AXIS_ORDERS = ("thw", "twh", "htw", "hwt", "wth", "wht")
+
+
+def reorder_tokens(x, perm, out=None, stream=None):
+    """x [B, H, L, d] with its rows gathered through perm ([L], or [B*H, L] per head) on the GPU."""
+    import torch
+    out = torch.empty_like(x) if out is None else out
+    C.pisa_permute_rows(x, out, perm, inverse=False, stream=stream)
+    return out
+
+
+def restore_tokens(x, perm, out=None, stream=None):
+    """Inverse of reorder_tokens: rows of x scattered back to their original positions."""
+    import torch
+    out = torch.empty_like(x) if out is None else out
+    C.pisa_permute_rows(x, out, perm, inverse=True, stream=stream)
+    return out
+
+
+def axis_order_permutations(grid, extra_tokens: int = 0, device="cuda"):
+    """Device int32 permutations [6, L] for the six axis orders of a (frames, height, width) grid."""
+    import torch
+    return torch.stack([torch.from_numpy(C.pisa_axis_permutation(grid, o, extra_tokens)) for o in AXIS_ORDERS]).to(device)
+
+
+def choose_axis_order(pisa: "Pisa", q, k, v, perms):
+    """Per head, the axis order whose blocks have the smallest total first-order spread sum_j M_j
+    (the method's own covariance measure, from the pre-computation on the reordered tokens).
+    Returns (per-head permutation [B*H, L] int32, chosen order index per head).  A calibration
+    step: six pre-computations."""
+    import torch
+    B, H = q.shape[0], q.shape[1]
+    scores = []
+    for r in range(perms.shape[0]):
+        qq, kk, vv = (reorder_tokens(x, perms[r]) for x in (q, k, v))
+        pisa.precompute(qq, kk, vv)
+        scores.append(pisa.stats.M.reshape(B * H, -1).sum(dim=1))
+    best = torch.stack(scores).argmin(dim=0)
+    return perms[best].contiguous(), best

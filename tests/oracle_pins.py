@@ -301,6 +301,59 @@ def pin_route_edges():
     return ok, f"tie sel {tsel}"
 
 
+# ---------------------------------------------------------------------------------------------
+# Token reordering pins ("PAROAttention: Pattern-Aware ReOrdering ...", abstract)
+# ---------------------------------------------------------------------------------------------
+def pin_axis_permutation_by_hand():
+    """A 2 x 2 x 3 grid listed as (h, w, t): t runs fastest, so positions alternate between the two
+    frames, 6 raster indices apart; identity for (t, h, w); extra tokens stay at the end."""
+    hwt = O.axis_permutation((2, 2, 3), "hwt")
+    want = [0, 6, 1, 7, 2, 8, 3, 9, 4, 10, 5, 11]          # written out from (h, w, t) = (0,0,0), (0,0,1), ...
+    ident = O.axis_permutation((2, 2, 3), "thw", extra_tokens=2)
+    wht = O.axis_permutation((1, 2, 2), "wht")
+    # gather semantics: row i of the output is row perm[i] of the input (rows labelled by index)
+    rows = O.permute_rows(np.arange(12.0)[:, None], hwt)[:, 0]
+    ok = (list(hwt) == want and list(ident) == list(range(14)) and list(wht) == [0, 2, 1, 3]
+          and list(rows) == want)
+    return ok, f"hwt {list(hwt)} rows {list(rows)}"
+
+
+def pin_axis_permutation_coordinates():
+    """Every order is a permutation, and consecutive positions step by one along the fastest axis."""
+    T, Hg, W = 3, 4, 5
+    ok = True
+    for order in ("thw", "twh", "htw", "hwt", "wth", "wht"):
+        perm = O.axis_permutation((T, Hg, W), order)
+        ok &= sorted(perm.tolist()) == list(range(T * Hg * W))
+        t, h, w = perm // (Hg * W), (perm // W) % Hg, perm % W
+        coord = {"t": t, "h": h, "w": w}
+        fast = coord[order[2]]
+        n_fast = {"t": T, "h": Hg, "w": W}[order[2]]
+        ok &= bool(np.all(fast == np.arange(T * Hg * W) % n_fast))
+    return ok, ""
+
+
+def pin_permute_rows_inverse_and_dense_equivariance():
+    """Scatter undoes gather; dense attention commutes with reordering the tokens (a property of
+    softmax attention, checked against torch SDPA): SDPA(Pq, Pk, Pv) = P SDPA(q, k, v)."""
+    q, k, v = _qkv(31, 60, 8)
+    perm = O.axis_permutation((3, 4, 5), "wht")
+    back = O.permute_rows(O.permute_rows(v, perm), perm, inverse=True)
+    lhs = _sdpa(O.permute_rows(q, perm), O.permute_rows(k, perm), O.permute_rows(v, perm), 0.7)
+    rhs = O.permute_rows(_sdpa(q, k, v, 0.7), perm)
+    e = _rel(lhs, rhs)
+    return np.array_equal(back, v) and e < 1e-12, f"rel {e:.2e}"
+
+
+def pin_reordered_pisa_all_selected_is_dense():
+    """PISA on reordered tokens with every block selected, put back in order = dense attention."""
+    q, k, v = _qkv(32, 60, 8)
+    perm = O.axis_permutation((3, 4, 5), "hwt")
+    r = O.pisa_reordered(q[None, None], k[None, None], v[None, None], perm, 16, 4, 0.5, 0.9)
+    e = _rel(r["o"][0, 0], _sdpa(q, k, v, 0.9))
+    return e < 1e-12, f"rel {e:.2e}"
+
+
 ALL_PINS = [
     pin_all_selected_is_dense, pin_block_one_is_dense, pin_constant_key_blocks_are_dense,
     pin_exact_only_is_masked_sdpa, pin_brute_force_matches, pin_value_shift_equivariance,
@@ -308,4 +361,6 @@ ALL_PINS = [
     pin_first_order_in_general, pin_block_means_and_sums, pin_first_order_matrix_is_cross_covariance,
     pin_global_statistic_closed_form, pin_cov_norm, pin_route_combination_rule, pin_route_count_weighting,
     pin_route_lambda_zero_is_pooled_topk, pin_route_large_lambda_is_cov_topk, pin_route_edges,
+    pin_axis_permutation_by_hand, pin_axis_permutation_coordinates,
+    pin_permute_rows_inverse_and_dense_equivariance, pin_reordered_pisa_all_selected_is_dense,
 ]

@@ -59,6 +59,20 @@ MUTATIONS["ties to the higher index"] = ("route_select", _tie_high)
 _ORIG["route_select"] = O.route_select
 
 
+def _axes_reversed(grid, order, extra_tokens=0):
+    return _ORIG["axis_permutation"](grid, order[::-1], extra_tokens)
+
+
+def _gather_is_scatter(x, perm, inverse=False):
+    return _ORIG["permute_rows"](x, perm, not inverse)
+
+
+MUTATIONS["axis order read fastest first"] = ("axis_permutation", _axes_reversed)
+MUTATIONS["gather and scatter swapped"] = ("permute_rows", _gather_is_scatter)
+_ORIG["axis_permutation"] = O.axis_permutation
+_ORIG["permute_rows"] = O.permute_rows
+
+
 def _caught():
     failed = []
     for pin in P.ALL_PINS:

@@ -39,6 +39,7 @@ __all__ = [
     "num_blocks", "block_bounds", "block_stats", "route_scores", "route_select",
     "attention_head", "pisa", "dense_attention", "brute_force_head",
     "axis_permutation", "permute_rows", "pisa_reordered",
+    "E4M3_MAX", "e4m3", "quantize_groups", "fp8_logit_inputs", "pisa_fp8",
 ]
 
 
@@ -178,11 +179,14 @@ def _denominator(ez: np.ndarray, alpha: np.ndarray, cnt_u: np.ndarray) -> np.nda
 
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, sel: np.ndarray,
                    stats: Dict, scale: float = 1.0, mode: str = "pisa",
-                   first_order: str = "global", qblocks: Optional[Sequence[int]] = None) -> np.ndarray:
+                   first_order: str = "global", qblocks: Optional[Sequence[int]] = None,
+                   q_corr: Optional[np.ndarray] = None) -> np.ndarray:
     """o = N / D for one head; ``mode='exact_only'`` drops U_i (the keep-or-drop baseline).
 
-    ``qblocks`` restricts the evaluation to those query blocks (other rows are NaN).
+    ``qblocks`` restricts the evaluation to those query blocks (other rows are NaN).  ``q_corr``,
+    when given, is the query used by the first-order correction (the logits use ``q``).
     """
+    qc_all = None if q_corr is None else np.asarray(q_corr, dtype=np.float64)
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -210,7 +214,8 @@ def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, block: int, sel:
         N = ez @ v[tok]                                               # exact sparse term
         if U:
             N = N + alpha @ stats["vsum"][U]                          # block-wise zeroth order
-            N = N + _correction(qi, stats, alpha, U, scale, first_order)
+            qc = qi if qc_all is None else qc_all[qs:qe]
+            N = N + _correction(qc, stats, alpha, U, scale, first_order)
         D = _denominator(ez, alpha, stats["cnt"][U] if U else np.zeros(0))
         o[qs:qe] = N / D[:, None]
     return o
@@ -354,3 +359,70 @@ def pisa_reordered(q, k, v, perm, block: int, keep_k: int, lam: float, scale: fl
     r = pisa(permute_rows(q, perm), permute_rows(k, perm), permute_rows(v, perm), block, keep_k, lam, scale, **kw)
     r["o"] = permute_rows(r["o"], perm, inverse=True)
     return r
+
+
+# --------------------------------------------------------------------------------------------
+# e4m3 logits for the exact stage (SURVEY's next row on low-bit attention, after PAROAttention's
+# INT8/INT4 remark in its abstract; the pages give no FP8 recipe, so this is a reading).  The
+# exact and zeroth-order logits use e4m3 copies of q (one scale per row), k (one scale per key
+# block) and kbar (one scale per tile of 128 centroids); the scale of a group is max|x| / 448 and
+# the code of x is e4m3(x / scale), both decided in float32.  Routing, the values and the
+# first-order correction keep the unquantized inputs.
+# --------------------------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3(x: np.ndarray) -> np.ndarray:
+    """Round float32 values (|x| <= 448) to the nearest e4m3 value, ties to even (torch's
+    float8_e4m3fn conversion on the CPU, a library primitive); returned as float64."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def quantize_groups(x: np.ndarray, group_of_row: np.ndarray):
+    """Per-group scale s_g = float32(max|x| over the group's rows) / 448 (1 for an all-zero group)
+    and dequantized values e4m3(x / s_g) * s_g.  Returns (dequantized float64, scales float32)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    ngroups = int(group_of_row.max()) + 1 if len(group_of_row) else 0
+    amax = np.zeros(ngroups, dtype=np.float32)
+    np.maximum.at(amax, group_of_row, np.abs(x32).max(axis=1))
+    sc = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    codes = e4m3((x32 / sc[group_of_row][:, None]).astype(np.float32))
+    return codes * sc[group_of_row][:, None].astype(np.float64), sc
+
+
+def fp8_logit_inputs(q: np.ndarray, k: np.ndarray, kbar: np.ndarray, block: int):
+    """Dequantized e4m3 copies of q (per row), k (per key block) and kbar (per 128 centroids)."""
+    L = q.shape[0]
+    nb = kbar.shape[0]
+    qd, _ = quantize_groups(q, np.arange(L))
+    kd, _ = quantize_groups(k, np.arange(L) // block)
+    kbd, _ = quantize_groups(kbar, np.arange(nb) // 128)
+    return qd, kd, kbd
+
+
+def pisa_fp8(q, k, v, block: int, keep_k: int, lam: float, scale: float = 1.0, mode: str = "pisa",
+             heads: Optional[Sequence[int]] = None, qblocks: Optional[Sequence[int]] = None) -> Dict:
+    """pisa() with the attention logits computed from the e4m3 copies (see above)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hh, L, d = q.shape
+    hs = list(range(Hh)) if heads is None else list(heads)
+    out: Dict[str, list] = {key: [] for key in ("o", "sel", "r")}
+    for b in range(B):
+        row = {key: [] for key in out}
+        for h in hs:
+            st = block_stats(q[b, h], k[b, h], v[b, h], block)
+            r = route_scores(st, lam, scale)
+            sel = route_select(r, keep_k)
+            qd, kd, kbd = fp8_logit_inputs(q[b, h], k[b, h], st["kbar"], block)
+            st_l = dict(st)
+            st_l["kbar"] = kbd
+            o = attention_head(qd, kd, v[b, h], block, sel, st_l, scale, mode, "global", qblocks, q_corr=q[b, h])
+            for key, val in (("o", o), ("sel", sel), ("r", r)):
+                row[key].append(val)
+        for key in out:
+            out[key].append(np.stack(row[key]))
+    return {key: np.stack(val) for key, val in out.items()}

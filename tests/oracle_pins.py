@@ -354,6 +354,76 @@ def pin_reordered_pisa_all_selected_is_dense():
     return e < 1e-12, f"rel {e:.2e}"
 
 
+# ---------------------------------------------------------------------------------------------
+# e4m3 logits (reading for the low-bit exact stage)
+# ---------------------------------------------------------------------------------------------
+def pin_e4m3_by_hand():
+    """e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals down to 2^-9, largest
+    finite 448) rounding to nearest, ties to even, worked out by hand from that definition."""
+    x = np.array([1.0, 1.0625, 1.1875, 0.1, 2.0 ** -9, 3 * 2.0 ** -10, 448.0, 447.9999, 240.0, 250.0, -3.3])
+    want = [1.0, 1.0, 1.25, 0.1015625, 2.0 ** -9, 2.0 ** -8, 448.0, 448.0, 240.0, 256.0, -3.25]
+    got = O.e4m3(x)
+    return bool(np.array_equal(got, want)), f"{got}"
+
+
+def pin_quantize_groups_bounds():
+    """Each group's largest |x| maps to the code 448; every value is within half a unit in the last
+    place (2^-4 relative, or 2^-10 * scale for subnormal codes)."""
+    x = _rng(40).standard_normal((12, 16)) * np.linspace(0.01, 5, 12)[:, None]
+    groups = np.arange(12) // 4
+    d, sc = O.quantize_groups(x, groups)
+    ok = True
+    for g in range(3):
+        rows = groups == g
+        big = np.abs(x[rows]).max()
+        ok &= abs(np.abs(d[rows]).max() - 448.0 * float(sc[g])) <= 1e-12 * big
+        ok &= abs(float(sc[g]) - np.float32(np.float32(big) / np.float32(448.0))) == 0.0
+        err = np.abs(d[rows] - x[rows])
+        ok &= bool(np.all(err <= 2.0 ** -4 * np.abs(x[rows]) + 2.0 ** -10 * float(sc[g]) + 1e-12))
+    return bool(ok), ""
+
+
+def _representable(r, n, d, scale_of_row, big_every=1):
+    """Rows of e4m3 codes times a per-row factor; every `big_every`-th row holds the code +-448
+    once, the others only smaller codes (so a group of big_every rows has its maximum in one row)."""
+    codes = np.array([1.0, 0.5, 2.0, 3.25, 96.0, 0.1015625, 13.0, 40.0, 1.75, 0.375])
+    x = r.choice(np.concatenate([codes, -codes]), size=(n, d))
+    big = np.arange(n) % big_every == 0
+    x[big, 0] = 448.0 * np.where(r.random(int(big.sum())) < 0.5, 1.0, -1.0)
+    return x * scale_of_row[:, None]
+
+
+def pin_fp8_exact_on_representable_inputs():
+    """q rows that are e4m3 codes times a row factor and key blocks that are codes times a block
+    factor quantize exactly (per-row q scales, per-block k scales): with every block selected the
+    e4m3-logit attention equals softmax attention (torch SDPA)."""
+    r = _rng(41)
+    L, d, block = 64, 8, 16
+    q = _representable(r, L, d, 0.003 * (1.0 + r.random(L)))
+    k = _representable(r, L, d, np.repeat(0.002 * (1.0 + r.random(L // block)), block), big_every=block)
+    v = r.standard_normal((L, d))
+    o = O.pisa_fp8(q[None, None], k[None, None], v[None, None], block, L // block, 0.5, 0.8)["o"][0, 0]
+    e = _rel(o, _sdpa(q, k, v, 0.8))
+    return e < 1e-6, f"rel {e:.2e}"
+
+
+def pin_fp8_constant_key_blocks_are_dense():
+    """Blocks of one constant, exactly representable key (the same factor for every block, so the
+    centroid tile quantizes exactly too): any keep_k gives softmax attention."""
+    r = _rng(42)
+    L, d, block = 64, 8, 16
+    q = _representable(r, L, d, 0.003 * (1.0 + r.random(L)))
+    c = _representable(r, L // block, d, np.full(L // block, 2.0 ** -8))
+    k = np.repeat(c, block, axis=0)
+    v = r.standard_normal((L, d))
+    dense = _sdpa(q, k, v, 0.8)
+    worst = 0.0
+    for keep in (0, 1, 4):
+        o = O.pisa_fp8(q[None, None], k[None, None], v[None, None], block, keep, 0.5, 0.8)["o"][0, 0]
+        worst = max(worst, _rel(o, dense))
+    return worst < 1e-6, f"rel {worst:.2e}"
+
+
 ALL_PINS = [
     pin_all_selected_is_dense, pin_block_one_is_dense, pin_constant_key_blocks_are_dense,
     pin_exact_only_is_masked_sdpa, pin_brute_force_matches, pin_value_shift_equivariance,
@@ -363,4 +433,6 @@ ALL_PINS = [
     pin_route_lambda_zero_is_pooled_topk, pin_route_large_lambda_is_cov_topk, pin_route_edges,
     pin_axis_permutation_by_hand, pin_axis_permutation_coordinates,
     pin_permute_rows_inverse_and_dense_equivariance, pin_reordered_pisa_all_selected_is_dense,
+    pin_e4m3_by_hand, pin_quantize_groups_bounds, pin_fp8_exact_on_representable_inputs,
+    pin_fp8_constant_key_blocks_are_dense,
 ]

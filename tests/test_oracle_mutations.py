@@ -73,6 +73,32 @@ _ORIG["axis_permutation"] = O.axis_permutation
 _ORIG["permute_rows"] = O.permute_rows
 
 
+def _k_per_row(q, k, kbar, block):
+    qd, _, kbd = _ORIG["fp8_logit_inputs"](q, k, kbar, block)
+    kd, _ = O.quantize_groups(k, np.arange(k.shape[0]))
+    return qd, kd, kbd
+
+
+def _q_per_block(q, k, kbar, block):
+    _, kd, kbd = _ORIG["fp8_logit_inputs"](q, k, kbar, block)
+    qd, _ = O.quantize_groups(q, np.arange(q.shape[0]) // block)
+    return qd, kd, kbd
+
+
+MUTATIONS["e4m3 k scaled per row"] = ("fp8_logit_inputs", _k_per_row)
+MUTATIONS["e4m3 q scaled per block"] = ("fp8_logit_inputs", _q_per_block)
+
+
+def _bf16_not_e4m3(x):
+    import torch
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+MUTATIONS["e4m3 rounding is bf16 rounding"] = ("e4m3", _bf16_not_e4m3)
+_ORIG["fp8_logit_inputs"] = O.fp8_logit_inputs
+_ORIG["e4m3"] = O.e4m3
+
+
 def _caught():
     failed = []
     for pin in P.ALL_PINS:

@@ -24,8 +24,9 @@
  *     has enqueued nothing and written nothing.
  *   - No exceptions cross the ABI.  The library keeps no mutable host state apart from a cache of
  *     device attributes and resolved driver entry points.
- *   - Supported on the GPU: dtype PISA_BF16 with head_dim 128 and block 64 or 128 (tensor-core
- *     path), and PISA_FP32 with head_dim 64 or 128 and block 64 or 128 (fp32 FMA path).
+ *   - Supported on the GPU: dtype PISA_BF16 or PISA_BF16_FP8QK with head_dim 128 and block 64 or
+ *     128 (tensor-core path), and PISA_FP32 with head_dim 64 or 128 and block 64 or 128 (fp32 FMA
+ *     path).
  */
 #ifndef PISA_H_
 #define PISA_H_
@@ -54,7 +55,14 @@ typedef enum {
   PISA_ERR_DEVICE_TIMEOUT = 4  /* a kernel's bounded wait ran out (reported by pisa_read_device_error) */
 } pisa_status;
 
-typedef enum { PISA_BF16 = 0, PISA_FP32 = 1 } pisa_dtype;
+/* PISA_BF16_FP8QK: q, k, v and o are bf16 as with PISA_BF16, but the attention logits (exact
+ * and zeroth order) are computed on the tensor core from e4m3 copies that pisa_precompute writes:
+ * q with one scale per row, k with one scale per key block, kbar with one scale per tile of 128
+ * centroids; a group's scale is max|x| / 448 and x's code is e4m3(x / scale), both in float32.
+ * Routing, the values and the first-order correction keep the bf16 / fp32 data.  A low-bit
+ * exact stage in the spirit of PAROAttention's INT8/INT4 attention (its abstract); the pages
+ * print no FP8 recipe.  head_dim 128 only; PISA_MODE_PER_BLOCK is not supported with it. */
+typedef enum { PISA_BF16 = 0, PISA_FP32 = 1, PISA_BF16_FP8QK = 2 } pisa_dtype;
 
 /* PISA_MODE_EXACT_ONLY drops U_i entirely (the keep-or-drop sparse attention the method is
  * compared against, §1 문제 정의); it needs keep_k >= 1.
@@ -95,6 +103,13 @@ typedef struct {
   float* vscale;   /* [B,H]            power of two >= max|v| / 256 (1 when max|v| <= 256)     */
   void*  hdiff_op; /* nullable bf16 [B,H,nb,d,d]: softmax_scale * (H_j - Hbar), row a = key dim;
                     * written only when non-null (PISA_BF16 and with_H); PISA_MODE_PER_BLOCK reads it */
+  /* PISA_BF16_FP8QK only (null otherwise): e4m3 codes (one byte each) and their float32 scales */
+  void*  q8;       /* e4m3 [B,H,L,d]        q / qscale[row]                                      */
+  void*  k8;       /* e4m3 [B,H,L,d]        k / kscale[block of the row]                         */
+  void*  kbar8;    /* e4m3 [B,H,nb,d]       kbar / kbscale[j / 128]                              */
+  float* qscale;   /* [B,H,L]               max_a |q_t,a| / 448 (1 for a zero row)               */
+  float* kscale;   /* [B,H,nb]              max over block j of |k| / 448                        */
+  float* kbscale;  /* [B,H,ceil(nb/128)]    max over the 128 centroids of a tile of |kbar| / 448 */
 } pisa_stats;
 
 /* ABI revision of this header. */

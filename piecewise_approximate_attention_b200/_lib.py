@@ -14,7 +14,7 @@ from typing import Optional
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libpisa_b200.so")
 
 PISA_OK, PISA_ERR_INVALID_ARG, PISA_ERR_UNSUPPORTED, PISA_ERR_CUDA, PISA_ERR_DEVICE_TIMEOUT = range(5)
-PISA_BF16, PISA_FP32 = 0, 1
+PISA_BF16, PISA_FP32, PISA_BF16_FP8QK = 0, 1, 2
 PISA_MODE_PISA, PISA_MODE_EXACT_ONLY, PISA_MODE_PER_BLOCK = 0, 1, 2
 PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 
@@ -33,7 +33,7 @@ class PisaShape(ctypes.Structure):
 class PisaStats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("qbar", "kbar", "vsum", "hbar", "M", "H", "kbar_op", "vsum_op", "hbar_op", "v_op", "vscale",
-                 "hdiff_op")]
+                 "hdiff_op", "q8", "k8", "kbar8", "qscale", "kscale", "kbscale")]
 
 
 class PisaError(RuntimeError):
@@ -103,7 +103,7 @@ def _stream(stream) -> Optional[int]:
 # Thin wrappers with the ABI's names
 # ---------------------------------------------------------------------------------------------
 def make_shape(batch, heads, seq_len, head_dim, block, dtype, softmax_scale=1.0) -> PisaShape:
-    dt = {"bf16": PISA_BF16, "fp32": PISA_FP32}.get(dtype, dtype)
+    dt = {"bf16": PISA_BF16, "fp32": PISA_FP32, "bf16_fp8qk": PISA_BF16_FP8QK}.get(dtype, dtype)
     return PisaShape(batch, heads, seq_len, head_dim, block, int(dt), float(softmax_scale))
 
 
@@ -143,6 +143,12 @@ class Stats:
     v_op: object
     vscale: object
     hdiff_op: Optional[object]
+    q8: Optional[object] = None          # e4m3 copies (uint8 views) and scales, PISA_BF16_FP8QK only
+    k8: Optional[object] = None
+    kbar8: Optional[object] = None
+    qscale: Optional[object] = None
+    kscale: Optional[object] = None
+    kbscale: Optional[object] = None
 
 
 def alloc_stats(shape: PisaShape, device, with_H: bool = False) -> Stats:
@@ -174,7 +180,10 @@ def alloc_stats(shape: PisaShape, device, with_H: bool = False) -> Stats:
                  view(st.H, f32, (B, H, nb, d, d)), view(st.kbar_op, bf, (B, H, nb, d)),
                  view(st.vsum_op, f16, (B, H, nb, d)), view(st.hbar_op, bf, (B, H, d, d)),
                  view(st.v_op, f16, (B, H, shape.seq_len, d)), view(st.vscale, f32, (B, H)),
-                 view(st.hdiff_op, bf, (B, H, nb, d, d)))
+                 view(st.hdiff_op, bf, (B, H, nb, d, d)), view(st.q8, torch.uint8, (B, H, shape.seq_len, d)),
+                 view(st.k8, torch.uint8, (B, H, shape.seq_len, d)), view(st.kbar8, torch.uint8, (B, H, nb, d)),
+                 view(st.qscale, f32, (B, H, shape.seq_len)), view(st.kscale, f32, (B, H, nb)),
+                 view(st.kbscale, f32, (B, H, (nb + 127) // 128)))
 
 
 def pisa_perblock_workspace_bytes(shape: PisaShape) -> int:

@@ -22,10 +22,10 @@ pisa_status check_shape(const pisa_shape* s, Dims* g) {
   if (!s) return PISA_ERR_INVALID_ARG;
   if (s->batch < 1 || s->heads < 1 || s->seq_len < 1 || s->head_dim < 1 || s->block < 1)
     return PISA_ERR_INVALID_ARG;
-  if (s->dtype != PISA_BF16 && s->dtype != PISA_FP32) return PISA_ERR_INVALID_ARG;
+  if (s->dtype != PISA_BF16 && s->dtype != PISA_FP32 && s->dtype != PISA_BF16_FP8QK) return PISA_ERR_INVALID_ARG;
   if (!std::isfinite(s->softmax_scale) || !(s->softmax_scale > 0.f)) return PISA_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
-  if (s->dtype == PISA_BF16 && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
+  if (bf16_inputs(s->dtype) && s->head_dim != 128) return PISA_ERR_UNSUPPORTED;
   if (s->block != 64 && s->block != 128) return PISA_ERR_UNSUPPORTED;
   const long long nb = ((long long)s->seq_len + s->block - 1) / s->block;
   if (nb > kMaxBlocks) return PISA_ERR_UNSUPPORTED;
@@ -47,9 +47,14 @@ pisa_status check_stats(const Dims& g, const pisa_stats* st, bool need_ops) {
   for (const void* p : req)
     if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
   if ((st->H && !aligned16(st->H)) || (st->hdiff_op && !aligned16(st->hdiff_op))) return PISA_ERR_INVALID_ARG;
-  if (need_ops && g.dtype == PISA_BF16) {
+  if (need_ops && bf16_inputs(g.dtype)) {
     const void* ops[] = {st->kbar_op, st->vsum_op, st->hbar_op, st->v_op, st->vscale};
     for (const void* p : ops)
+      if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
+  }
+  if (need_ops && g.dtype == PISA_BF16_FP8QK) {
+    const void* f8[] = {st->q8, st->k8, st->kbar8, st->qscale, st->kscale, st->kbscale};
+    for (const void* p : f8)
       if (!p || !aligned16(p)) return PISA_ERR_INVALID_ARG;
   }
   return PISA_OK;
@@ -59,12 +64,13 @@ pisa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PISA_OK : PIS
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-constexpr int kStatsArrays = 12;
+constexpr int kStatsArrays = 18;
 
 // Sizes of the stats arrays in carve order.
 void stats_sizes(const Dims& g, int with_H, size_t out[kStatsArrays]) {
   const size_t bh = (size_t)g.BH(), nb = (size_t)g.nb, d = (size_t)g.d;
-  const bool ops = g.dtype == PISA_BF16;
+  const bool ops = bf16_inputs(g.dtype);
+  const bool f8 = g.dtype == PISA_BF16_FP8QK;
   out[0] = bh * nb * d * 4;            // qbar
   out[1] = bh * nb * d * 4;            // kbar
   out[2] = bh * nb * d * 4;            // vsum
@@ -77,6 +83,12 @@ void stats_sizes(const Dims& g, int with_H, size_t out[kStatsArrays]) {
   out[9] = ops ? bh * (size_t)g.L * d * 2 : 0;   // v_op
   out[10] = ops ? bh * 4 : 0;          // vscale
   out[11] = (ops && with_H) ? bh * nb * d * d * 2 : 0;   // hdiff_op
+  out[12] = f8 ? bh * (size_t)g.L * d : 0;               // q8
+  out[13] = f8 ? bh * (size_t)g.L * d : 0;               // k8
+  out[14] = f8 ? bh * nb * d : 0;                        // kbar8
+  out[15] = f8 ? bh * (size_t)g.L * 4 : 0;               // qscale
+  out[16] = f8 ? bh * nb * 4 : 0;                        // kscale
+  out[17] = f8 ? bh * ((nb + 127) / 128) * 4 : 0;        // kbscale
 }
 
 }  // namespace
@@ -86,7 +98,7 @@ using namespace pisa;
 
 extern "C" {
 
-int32_t pisa_abi_version(void) { return 3; }
+int32_t pisa_abi_version(void) { return 4; }
 
 int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
   if (seq_len < 1 || block < 1) return -1;
@@ -130,6 +142,12 @@ pisa_status pisa_stats_carve(const pisa_shape* shape, void* base, size_t bytes, 
   st.v_op = ptr[9];
   st.vscale = static_cast<float*>(ptr[10]);
   st.hdiff_op = ptr[11];
+  st.q8 = ptr[12];
+  st.k8 = ptr[13];
+  st.kbar8 = ptr[14];
+  st.qscale = static_cast<float*>(ptr[15]);
+  st.kscale = static_cast<float*>(ptr[16]);
+  st.kbscale = static_cast<float*>(ptr[17]);
   *out = st;
   return PISA_OK;
 }
@@ -160,7 +178,11 @@ pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* 
   if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
   if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (g.dtype == PISA_BF16) return cuda_status(launch_precompute_sm100(g, q, k, v, *stats, ws, cs));
+  if (bf16_inputs(g.dtype)) {
+    cudaError_t e = launch_precompute_sm100(g, q, k, v, *stats, ws, cs);
+    if (e == cudaSuccess && g.dtype == PISA_BF16_FP8QK) e = launch_quantize_fp8(g, q, k, *stats, cs);
+    return cuda_status(e);
+  }
   return cuda_status(launch_precompute_simt(g, q, k, v, *stats, ws, cs));
 }
 
@@ -192,13 +214,14 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
   if (keep_k > 0 && (!sel || !aligned16(sel))) return PISA_ERR_INVALID_ARG;
   if (order && !aligned16(order)) return PISA_ERR_INVALID_ARG;
   if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
+  if (mode == PISA_MODE_PER_BLOCK && g.dtype == PISA_BF16_FP8QK) return PISA_ERR_UNSUPPORTED;
   if (mode == PISA_MODE_PER_BLOCK && !(g.dtype == PISA_BF16 ? stats->hdiff_op : stats->H)) return PISA_ERR_INVALID_ARG;
   if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   const bool per_block = mode == PISA_MODE_PER_BLOCK && keep_k < g.nb;
   if (per_block && g.dtype == PISA_BF16 && ws_bytes < pisa_perblock_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   int* status = static_cast<int*>(ws);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (g.dtype == PISA_BF16) {
+  if (bf16_inputs(g.dtype)) {
     AttnMaps maps;
     const uint64_t bh = (uint64_t)g.BH();
     if (!encode_bf16_3d(&maps.q, q, g.d, g.L, bh, g.block) || !encode_bf16_3d(&maps.k, k, g.d, g.L, bh, g.block) ||
@@ -207,6 +230,16 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
         !encode_16bit_3d(&maps.vsum, stats->vsum_op, g.d, g.nb, bh, 128, true) ||
         !encode_bf16_3d(&maps.hbar, stats->hbar_op, g.d, g.d, bh, 128))
       return PISA_ERR_CUDA;
+    F8Scales f8;
+    if (g.dtype == PISA_BF16_FP8QK) {
+      if (!encode_u8_3d(&maps.q8, stats->q8, g.d, g.L, bh, g.block) ||
+          !encode_u8_3d(&maps.k8, stats->k8, g.d, g.L, bh, g.block) ||
+          !encode_u8_3d(&maps.kbar8, stats->kbar8, g.d, g.nb, bh, 128))
+        return PISA_ERR_CUDA;
+      f8.q = stats->qscale;
+      f8.k = stats->kscale;
+      f8.kb = stats->kbscale;
+    }
     const unsigned long long wait_ns = g_test_wait_ns ? g_test_wait_ns : kWaitLimitNs;
     // per-block mode: the attention kernel runs in PISA mode, leaves each row's softmax offset and
     // 1/D_t and its fp32 output in ws; the second kernel adds the per-block minus global first-order
@@ -215,7 +248,7 @@ pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k
     float2* rows = per_block ? reinterpret_cast<float2*>(wsb + kStatusBytes) : nullptr;
     float* o32 = per_block ? reinterpret_cast<float*>(wsb + o32_offset(g)) : nullptr;
     cudaError_t e = launch_attention_sm100(g, maps, sel, order, keep_k, mode == PISA_MODE_EXACT_ONLY ? mode : PISA_MODE_PISA,
-                                           stats->vscale, o, rows, o32, status, wait_ns, g_test_fault, cs);
+                                           stats->vscale, f8, o, rows, o32, status, wait_ns, g_test_fault, cs);
     if (e != cudaSuccess || !per_block) return cuda_status(e);
     CUtensorMap hmap;
     if (!encode_bf16_3d(&hmap, stats->hdiff_op, g.d, (uint64_t)g.nb * g.d, bh, 128)) return PISA_ERR_CUDA;

@@ -61,6 +61,7 @@ struct alignas(1024) Smem {
   uint64_t bar_kfull[kKS], bar_kempty[kKS], bar_vfull[kVS], bar_vempty[kVS];
   uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2];
   uint64_t bar_q, bar_final, bar_drain;
+  uint64_t bar_q16;          // e4m3 logits: the bf16 Q tile for the correction, loaded at the end
   uint32_t tmem_base;
   int abort;
   int n_exact, n_cent, need_corr;
@@ -76,6 +77,9 @@ struct Params {
   int fault;                 // test-only fault injection (pisa_testing.h); 0 in normal calls
   const int32_t* sel;
   const int32_t* order;
+  const float* qscale;       // e4m3 logits only: per-row, per-key-block and per-centroid-tile scales
+  const float* kscale;
+  const float* kbscale;
   __nv_bfloat16* o;
   float2* rowstats;          // nullable [B*H][L]: (softmax offset m*s*log2(e), 1/D_t) per row
   float* o32;                // nullable [B*H][L][D]: the output in fp32 instead of bf16 in o
@@ -152,6 +156,10 @@ __device__ void build_bits(uint32_t* bits, const Params& p, int bh, int qi) {
   }
 }
 
+// kF8: logits from e4m3 copies of q, k and kbar (kind::f8f6f4 MMAs, K = 32 per instruction); each
+// half's raw scores are scaled by its row's q scale times the key block's (or centroid tile's) k
+// scale before they enter the max and the exponent.  The correction keeps the bf16 Q tile.
+template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -195,6 +203,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     }
     mbar_init(&sm.bar_final, 1);
     mbar_init(&sm.bar_drain, 1);
+    mbar_init(&sm.bar_q16, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -233,16 +242,22 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
       if (p.fault != 1) {      // fault 1 (tests only): never load Q, so the MMA warp's wait runs out
-        mbar_expect_tx(&sm.bar_q, kTileBytes);
-        tma_load_3d(sm.q, &maps.q, &sm.bar_q, 0, qa * p.block, bh);
-        tma_load_3d(sm.q + kHalf, &maps.q, &sm.bar_q, 64, qa * p.block, bh);
-        if (pair) {
-          tma_load_3d(sm.q + 64 * 128, &maps.q, &sm.bar_q, 0, qb * p.block, bh);
-          tma_load_3d(sm.q + kHalf + 64 * 128, &maps.q, &sm.bar_q, 64, qb * p.block, bh);
+        if (kF8) {             // e4m3 Q: one 128-byte row per token, 16 KB
+          mbar_expect_tx(&sm.bar_q, kHalf);
+          tma_load_3d(sm.q, &maps.q8, &sm.bar_q, 0, qa * p.block, bh);
+          if (pair) tma_load_3d(sm.q + 64 * 128, &maps.q8, &sm.bar_q, 0, qb * p.block, bh);
+        } else {
+          mbar_expect_tx(&sm.bar_q, kTileBytes);
+          tma_load_3d(sm.q, &maps.q, &sm.bar_q, 0, qa * p.block, bh);
+          tma_load_3d(sm.q + kHalf, &maps.q, &sm.bar_q, 64, qa * p.block, bh);
+          if (pair) {
+            tma_load_3d(sm.q + 64 * 128, &maps.q, &sm.bar_q, 0, qb * p.block, bh);
+            tma_load_3d(sm.q + kHalf + 64 * 128, &maps.q, &sm.bar_q, 64, qb * p.block, bh);
+          }
         }
       }
       UnionIter it;
-      int issued_k = 0, issued_v = 0;
+      int issued_k = 0, issued_v = 0, issued_q16 = 0;
       bool ok = true;
       for (int t = 0; t < T && ok; ++t) {
         const int ks = t % kKS, vs = t % kVS;
@@ -251,20 +266,34 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         const int j1 = kt.j1 >= 0 ? kt.j1 : kt.j0;     // absent second block: reload the first, masked
         uint8_t* kb = sm.k[ks];
         uint64_t* kf = &sm.bar_kfull[ks];
-        mbar_expect_tx(kf, kTileBytes);
-        if (kt.kind == 0) {
-          if (pair) {
-            tma_load_3d(kb, &maps.k, kf, 0, kt.j0 * 64, bh);
-            tma_load_3d(kb + kHalf, &maps.k, kf, 64, kt.j0 * 64, bh);
-            tma_load_3d(kb + 64 * 128, &maps.k, kf, 0, j1 * 64, bh);
-            tma_load_3d(kb + kHalf + 64 * 128, &maps.k, kf, 64, j1 * 64, bh);
+        if (kF8) {               // e4m3 keys or centroids: 128 rows of 128 bytes
+          mbar_expect_tx(kf, kHalf);
+          if (kt.kind == 0) {
+            if (pair) {
+              tma_load_3d(kb, &maps.k8, kf, 0, kt.j0 * 64, bh);
+              tma_load_3d(kb + 64 * 128, &maps.k8, kf, 0, j1 * 64, bh);
+            } else {
+              tma_load_3d(kb, &maps.k8, kf, 0, kt.j0 * 128, bh);
+            }
           } else {
-            tma_load_3d(kb, &maps.k, kf, 0, kt.j0 * 128, bh);
-            tma_load_3d(kb + kHalf, &maps.k, kf, 64, kt.j0 * 128, bh);
+            tma_load_3d(kb, &maps.kbar8, kf, 0, kt.j0, bh);
           }
         } else {
-          tma_load_3d(kb, &maps.kbar, kf, 0, kt.j0, bh);
-          tma_load_3d(kb + kHalf, &maps.kbar, kf, 64, kt.j0, bh);
+          mbar_expect_tx(kf, kTileBytes);
+          if (kt.kind == 0) {
+            if (pair) {
+              tma_load_3d(kb, &maps.k, kf, 0, kt.j0 * 64, bh);
+              tma_load_3d(kb + kHalf, &maps.k, kf, 64, kt.j0 * 64, bh);
+              tma_load_3d(kb + 64 * 128, &maps.k, kf, 0, j1 * 64, bh);
+              tma_load_3d(kb + kHalf + 64 * 128, &maps.k, kf, 64, j1 * 64, bh);
+            } else {
+              tma_load_3d(kb, &maps.k, kf, 0, kt.j0 * 128, bh);
+              tma_load_3d(kb + kHalf, &maps.k, kf, 64, kt.j0 * 128, bh);
+            }
+          } else {
+            tma_load_3d(kb, &maps.kbar, kf, 0, kt.j0, bh);
+            tma_load_3d(kb + kHalf, &maps.kbar, kf, 64, kt.j0, bh);
+          }
         }
         ++issued_k;
         if (t >= kVS && !(ok = wait_or_abort(sm, &sm.bar_vempty[vs], ((t / kVS) - 1) & 1, p))) break;
@@ -295,12 +324,28 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           tma_load_3d(sm.k[ks] + kHalf, &maps.hbar, &sm.bar_kfull[ks], 64, 0, bh);
           ++issued_k;
         }
+        if (kF8 && ok) {
+          // the correction multiplies the bf16 Q tile: into the value buffer once the last PV is done
+          const int vs = T % kVS;
+          if (T < kVS || (ok = wait_or_abort(sm, &sm.bar_vempty[vs], ((T / kVS) - 1) & 1, p))) {
+            mbar_expect_tx(&sm.bar_q16, kTileBytes);
+            tma_load_3d(sm.v[vs], &maps.q, &sm.bar_q16, 0, qa * p.block, bh);
+            tma_load_3d(sm.v[vs] + kHalf, &maps.q, &sm.bar_q16, 64, qa * p.block, bh);
+            if (pair) {
+              tma_load_3d(sm.v[vs] + 64 * 128, &maps.q, &sm.bar_q16, 0, qb * p.block, bh);
+              tma_load_3d(sm.v[vs] + kHalf + 64 * 128, &maps.q, &sm.bar_q16, 64, qb * p.block, bh);
+            }
+            issued_q16 = 1;
+          }
+        }
       }
       {
         // drain: every copy issued must land before this CTA's shared memory is released (in a
         // normal run the MMA warp has waited for all of them, so these waits return at once)
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
+        if (issued_q16)
+          while (!mbar_try_wait(&sm.bar_q16, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
         for (int i = max(0, issued_k - kKS); i < issued_k; ++i)
           while (!mbar_try_wait(&sm.bar_kfull[i % kKS], (i / kKS) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
         for (int i = max(0, issued_v - kVS); i < issued_v; ++i)
@@ -328,10 +373,17 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           tc_fence_after();
         }
         const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ks]) + 8192 * hh, 16, 1024);
+        if (kF8) {
+          // e4m3 rows are 128 bytes: the four K = 32 steps are 32-byte column offsets of one row
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;   // start-address field units
-          mma_ss(tmem + kColS + 64 * hh, qd + off, kd + off, idesc_s, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss_f8(tmem + kColS + 64 * hh, qd + (kk * 32 >> 4), kd + (kk * 32 >> 4), idesc_e4m3_f32(128, 64), kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;   // start-address field units
+            mma_ss(tmem + kColS + 64 * hh, qd + off, kd + off, idesc_s, kk > 0);
+          }
         }
         mma_commit(&sm.bar_sfull[hh]);
         if (hh == 1) mma_commit(&sm.bar_kempty[ks]);
@@ -362,13 +414,16 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       if (ok && need_corr) {
         // Q (s Hbar^T) into columns 0..127, after every PV has read its P there
         const int ks = T % kKS;
-        if ((ok = wait_or_abort(sm, &sm.bar_kfull[ks], (T / kKS) & 1, p))) {
+        // with e4m3 logits the correction's A operand is the bf16 Q tile loaded into the value buffer
+        if ((ok = wait_or_abort(sm, &sm.bar_kfull[ks], (T / kKS) & 1, p)) &&
+            (!kF8 || (ok = wait_or_abort(sm, &sm.bar_q16, 0, p)))) {
           tc_fence_after();
           const uint64_t kd = smem_desc_sw128(smem_u32(sm.k[ks]), 16, 1024);
+          const uint64_t ad = kF8 ? smem_desc_sw128(smem_u32(sm.v[T % kVS]), 16, 1024) : qd;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = ((kk >> 2) * kHalf + (kk & 3) * 32) >> 4;
-            mma_ss(tmem + kColS, qd + off, kd + off, idesc_c, kk > 0);
+            mma_ss(tmem + kColS, ad + off, kd + off, idesc_c, kk > 0);
           }
         }
       }
@@ -392,15 +447,30 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
     const bool row_valid = rloc < block_count(myq, p.L, p.block) && (!upper || has_b);
     const float last_cnt = (float)block_count(p.nb - 1, p.L, p.block);
     float m = -INFINITY, l = 0.f, A = 0.f;
+    // e4m3 logits: this row's q scale, and the k scales of the current tile's two halves
+    const float qsc = (kF8 && row_valid) ? p.qscale[(size_t)bh * p.L + (size_t)myq * p.block + rloc] : 1.f;
+    float ksc0 = 1.f, ksc1 = 1.f;
     UnionIter it;
     KeyTile kt{0, 0, -1};
     bool ok = true;
     for (int u = 0; u < 2 * T; ++u) {
       const int t = u >> 1, hh = u & 1;
+      if (hh == 0) {
+        kt = key_tile(t, n_exact, pair, it, sm.bitsA, sm.bitsB);
+        if (kF8) {   // issued before the wait, so the loads overlap it
+          const size_t kb0 = (size_t)bh * p.nb;
+          if (kt.kind == 1) {
+            ksc0 = ksc1 = p.kbscale[(size_t)bh * ((p.nb + 127) / 128) + (kt.j0 >> 7)];
+          } else {
+            ksc0 = p.kscale[kb0 + kt.j0];
+            ksc1 = pair ? (kt.j1 >= 0 ? p.kscale[kb0 + kt.j1] : 1.f) : ksc0;
+          }
+        }
+      }
       ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_sfull[hh], t & 1, p));
       if (!ok) break;
       tc_fence_after();
-      if (hh == 0) kt = key_tile(t, n_exact, pair, it, sm.bitsA, sm.bitsB);
+      const float sl = kF8 ? qsc * (hh ? ksc1 : ksc0) : 1.f;   // raw MMA score -> logit
       const bool centroid = kt.kind == 1;
       float s[64];
       tmem_ld32(trow + kColS + 64 * hh, s);
@@ -436,7 +506,8 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         t2 = fmax3(t2, s[c + 4], s[c + 5]);
         t3 = fmax3(t3, s[c + 6], s[c + 7]);
       }
-      const float m_new = fmaxf(m, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));   // raw logit units
+      const float hmax = fmaxf(fmaxf(t0, t1), fmaxf(t2, t3));
+      const float m_new = fmaxf(m, kF8 ? hmax * sl : hmax);   // logit units
       const bool grow = m_new > m + p.lazy;
       const float f = grow ? ex2((m - m_new) * p.scale_log2) : 1.f;   // 0 when m = -inf
       if (grow) {
@@ -454,7 +525,8 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       // p = 2^(s*scale*log2e - m*scale*log2e) (masked entries are -inf and give exactly 0), two at a
       // time with f32x2 arithmetic; P (bf16) goes over the first 32 columns of this half's S
       const float mb = m == -INFINITY ? 0.f : m * p.scale_log2;
-      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nmb2 = f2_pack(-mb, -mb);
+      const float scl = kF8 ? p.scale_log2 * sl : p.scale_log2;
+      const uint64_t sc2 = f2_pack(scl, scl), nmb2 = f2_pack(-mb, -mb);
       uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
@@ -477,7 +549,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         // alpha of every unselected block enters D with weight cnt_j: `block` except the last one
         A += ls;
         l = fmaf((float)p.block, ls, l);
-        if (has_last) l = fmaf(last_cnt - (float)p.block, ex2(fmaf(slast, p.scale_log2, -mb)), l);
+        if (has_last) l = fmaf(last_cnt - (float)p.block, ex2(fmaf(slast, scl, -mb)), l);
       } else {
         l += ls;
       }
@@ -560,8 +632,8 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
 size_t attention_sm100_smem_bytes() { return sizeof(Smem) + 1024; }
 
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
-                                   int keep_k, int mode, const float* vscale, void* o, float2* rowstats,
-                                   float* o32, int* status, unsigned long long wait_ns, int fault,
+                                   int keep_k, int mode, const float* vscale, const F8Scales& f8, void* o,
+                                   float2* rowstats, float* o32, int* status, unsigned long long wait_ns, int fault,
                                    cudaStream_t stream) {
   Params p;
   p.L = g.L;
@@ -576,6 +648,9 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
   p.fault = fault;
   p.sel = sel;
   p.order = order;
+  p.qscale = f8.q;
+  p.kscale = f8.k;
+  p.kbscale = f8.kb;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.rowstats = rowstats;
   p.o32 = o32;
@@ -583,9 +658,14 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
   p.wait_ns = wait_ns;
   const size_t smem = attention_sm100_smem_bytes();
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(attn_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
   const int ntiles = g.block == 64 ? (g.nb + 1) / 2 : g.nb;
-  attn_sm100<<<dim3(ntiles, g.BH()), kThreads, smem, stream>>>(maps, p);
+  if (f8.q) {
+    if ((e = cudaFuncSetAttribute(attn_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+    attn_sm100<true><<<dim3(ntiles, g.BH()), kThreads, smem, stream>>>(maps, p);
+  } else {
+    if ((e = cudaFuncSetAttribute(attn_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+    attn_sm100<false><<<dim3(ntiles, g.BH()), kThreads, smem, stream>>>(maps, p);
+  }
   return cudaGetLastError();
 }
 

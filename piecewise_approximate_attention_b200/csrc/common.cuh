@@ -54,9 +54,21 @@ __device__ __forceinline__ int block_count(int j, int L, int block) {
   return e - s;
 }
 
-// TMA descriptors of one pisa_attention call (bf16 path).
+// Inputs stored as bf16 (PISA_BF16, and PISA_BF16_FP8QK whose logits use e4m3 copies).
+inline bool bf16_inputs(int dtype) { return dtype == PISA_BF16 || dtype == PISA_BF16_FP8QK; }
+
+// TMA descriptors of one pisa_attention call (bf16 inputs); q8, k8, kbar8 only for e4m3 logits.
 struct AttnMaps {
   CUtensorMap q, k, v, kbar, vsum, hbar;
+  CUtensorMap q8, k8, kbar8;
+};
+
+// Scales of the e4m3 operand copies (all null on the bf16 path): per query row [B*H][L], per key
+// block [B*H][nb], per tile of 128 centroids [B*H][ceil(nb/128)].
+struct F8Scales {
+  const float* q = nullptr;
+  const float* k = nullptr;
+  const float* kb = nullptr;
 };
 
 // Encodes a 3-D bf16 tensor [batch][rows][inner] (row-major) with a {64, box_rows, 1} box and
@@ -66,6 +78,9 @@ bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
 // Same for a bf16 (fp16 == false) or fp16 (fp16 == true) tensor.
 bool encode_16bit_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
                      uint32_t box_rows, bool fp16);
+// A 3-D byte tensor [batch][rows][128] with a {128, box_rows, 1} box and 128-byte swizzling (e4m3).
+bool encode_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                  uint32_t box_rows);
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits: 2 s
 
@@ -79,9 +94,10 @@ cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts,
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream);
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
-                                   int keep_k, int mode, const float* vscale, void* o, float2* rowstats,
-                                   float* o32, int* status, unsigned long long wait_ns, int fault,
+                                   int keep_k, int mode, const float* vscale, const F8Scales& f8, void* o,
+                                   float2* rowstats, float* o32, int* status, unsigned long long wait_ns, int fault,
                                    cudaStream_t stream);
+cudaError_t launch_quantize_fp8(const Dims& g, const void* q, const void* k, const pisa_stats& st, cudaStream_t stream);
 cudaError_t launch_permute_rows(const void* src, void* dst, const int32_t* perm, int batch_heads, int L,
                                 int row_bytes, int perm_per_head, int inverse, cudaStream_t stream);
 cudaError_t launch_perblock_sm100(const Dims& g, const AttnMaps& maps, const CUtensorMap& hdiff,

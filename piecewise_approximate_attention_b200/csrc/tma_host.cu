@@ -43,4 +43,18 @@ bool encode_16bit_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
   return r == CUDA_SUCCESS;
 }
 
+bool encode_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                  uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn || !base || inner != 128) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner, rows * inner};
+  cuuint32_t box[3] = {128, box_rows, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace pisa

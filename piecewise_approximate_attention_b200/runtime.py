@@ -25,7 +25,8 @@ class Pisa:
         self.block, self.keep_k, self.lam, self.mode = block, keep_k, lam, mode
         self.nb = C.pisa_num_blocks(seq_len, block)
         self.device = torch.device(device)
-        self.tdtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.tdtype = torch.float32 if dtype == "fp32" else torch.bfloat16
+        self.fp8 = dtype == "bf16_fp8qk"
         self._torch_f32 = torch.float32
         if mode == C.PISA_MODE_PER_BLOCK:
             with_H = True         # the per-block first-order matrices live in the stats
@@ -74,11 +75,11 @@ class Pisa:
         return graph
 
     def launches_per_step(self) -> int:
-        """Kernels one __call__ enqueues: pre-compute 3, routing 1 (+1 pairing), attention 1 (+1 for
-        the per-block first-order kernel on the bf16 path)."""
+        """Kernels one __call__ enqueues: pre-compute 3 (+3 e4m3 quantizations), routing 1 (+1
+        pairing), attention 1 (+1 for the per-block first-order kernel on the bf16 path)."""
         extra = 1 if (self.mode == C.PISA_MODE_PER_BLOCK and self.tdtype != self._torch_f32 and
                       self.keep_k < self.nb) else 0
-        return 3 + 1 + (1 if self.order is not None else 0) + 1 + extra
+        return 3 + (3 if self.fp8 else 0) + 1 + (1 if self.order is not None else 0) + 1 + extra
 
     def device_error(self, stream=None):
         return C.pisa_read_device_error(self.ws, stream)

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_blocks():
-    assert C.lib().pisa_abi_version() == 3
+    assert C.lib().pisa_abi_version() == 4
     assert C.pisa_num_blocks(32760, 64) == 512
     assert C.pisa_num_blocks(75600, 128) == 591
     assert C.pisa_num_blocks(1, 64) == 1
@@ -79,6 +79,15 @@ def test_stats_bytes_and_carve_are_host_only():
     n32h = C.pisa_stats_bytes(f32, True)
     assert C.lib().pisa_stats_carve(ctypes.byref(f32), base, n32h, 1, ctypes.byref(st32)) == C.PISA_OK
     assert st32.H and not st32.hdiff_op
+    assert not st0.q8 and not st0.qscale
+    # e4m3 logits: operand copies plus the e4m3 copies and their scales
+    f8 = _shape(dtype="bf16_fp8qk")
+    n8 = C.pisa_stats_bytes(f8, False)
+    st8 = C.PisaStats()
+    assert C.lib().pisa_stats_carve(ctypes.byref(f8), base, n8, 0, ctypes.byref(st8)) == C.PISA_OK
+    f8ptrs = [st8.q8, st8.k8, st8.kbar8, st8.qscale, st8.kscale, st8.kbscale, st8.kbar_op, st8.v_op]
+    assert all(p and p % 256 == 0 for p in f8ptrs) and len(set(f8ptrs)) == len(f8ptrs)
+    assert n8 - n0 >= 2 * 2 * 1000 * 128 + 2 * 16 * 128 + 2 * 1000 * 4
 
 
 @pytest.mark.parametrize("kw,expect", [
@@ -91,6 +100,8 @@ def test_stats_bytes_and_carve_are_host_only():
     (dict(softmax_scale=0.0), C.PISA_ERR_INVALID_ARG),
     (dict(softmax_scale=-1.0), C.PISA_ERR_INVALID_ARG),
     (dict(seq_len=64 * 4097), C.PISA_ERR_UNSUPPORTED),
+    (dict(dtype=3), C.PISA_ERR_INVALID_ARG),
+    (dict(dtype="bf16_fp8qk", head_dim=64), C.PISA_ERR_UNSUPPORTED),
 ])
 def test_bad_shapes_rejected(kw, expect):
     sh = _shape(**kw)
@@ -150,6 +161,18 @@ def test_invalid_arguments_rejected_without_launch():
     assert att(4, C.PISA_MODE_PISA, wsb=100) == C.PISA_ERR_INVALID_ARG
     code = ctypes.c_int32()
     assert L.pisa_read_device_error(None, ctypes.byref(code), None) == C.PISA_ERR_INVALID_ARG
+    # e4m3 logits need their copies in the stats, and do not combine with the per-block mode
+    f8 = _shape(dtype="bf16_fp8qk")
+    st8 = _fake_stats(f8)
+    b8 = ctypes.byref(f8)
+    ws8 = C.pisa_perblock_workspace_bytes(f8)
+    assert L.pisa_attention(b8, P, P, P, ctypes.byref(st8), P, None, 4, C.PISA_MODE_PER_BLOCK, P, P, ws8,
+                            None) == C.PISA_ERR_UNSUPPORTED
+    bad8 = C.PisaStats.from_buffer_copy(st8)
+    bad8.kscale = None
+    assert L.pisa_attention(b8, P, P, P, ctypes.byref(bad8), P, None, 4, C.PISA_MODE_PISA, P, P, ws8,
+                            None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_precompute(b8, P, P, P, ctypes.byref(bad8), P, ws8, None) == C.PISA_ERR_INVALID_ARG
 
 
 def test_missing_library_fails_loudly(monkeypatch):

@@ -12,6 +12,7 @@ namespace pisa {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
 
 __global__ void __launch_bounds__(kThreads) permute_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                                 const int32_t* __restrict__ perm, int L,
@@ -20,13 +21,30 @@ __global__ void __launch_bounds__(kThreads) permute_rows_kernel(const uint4* __r
   const int bh = blockIdx.y;
   const int32_t* pr = perm + (perm_per_head ? (size_t)bh * L : 0);
   const size_t base = (size_t)bh * L * chunks;
-  for (long long e = (long long)blockIdx.x * kThreads + threadIdx.x; e < total; e += (long long)gridDim.x * kThreads) {
-    const int i = (int)(e / chunks), c = (int)(e % chunks);
-    const int j = pr[i];
-    if (j < 0 || j >= L) continue;   // out-of-range entries are skipped (documented in pisa.h)
-    const size_t from = inverse ? (size_t)i : (size_t)j;
-    const size_t to = inverse ? (size_t)j : (size_t)i;
-    dst[base + to * chunks + c] = src[base + from * chunks + c];
+  const long long stride = (long long)gridDim.x * kThreads;
+  // kUnroll chunks per thread per round: all loads are issued before the stores
+  for (long long e0 = (long long)blockIdx.x * kThreads + threadIdx.x; e0 < total; e0 += kUnroll * stride) {
+    uint4 val[kUnroll];
+    size_t to[kUnroll];
+    bool ok[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long e = e0 + u * stride;
+      ok[u] = false;
+      if (e < total) {
+        const int i = (int)(e / chunks), c = (int)(e % chunks);
+        const int j = pr[i];
+        if (j >= 0 && j < L) {   // out-of-range entries are skipped (documented in pisa.h)
+          const size_t from = inverse ? (size_t)i : (size_t)j;
+          to[u] = base + (inverse ? (size_t)j : (size_t)i) * chunks + c;
+          val[u] = src[base + from * chunks + c];
+          ok[u] = true;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (ok[u]) dst[to[u]] = val[u];
   }
 }
 

@@ -290,6 +290,9 @@ struct alignas(1024) SmemB {
   int abort;
 };
 
+// kDiff: also write the per-block first-order operand copy s (H_j - Hbar) (stats with H only); a
+// template parameter so that the usual pass keeps its registers for the norms.
+template <bool kDiff>
 __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_constant__ KVMaps maps, const PreParams p) {
   extern __shared__ uint8_t smem_raw[];
   SmemB& sm = *reinterpret_cast<SmemB*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
         bar_epi();
         float ss = 0.f;
         float* Hout = (live && p.st.H) ? p.st.H + ((size_t)bh * p.nb + j) * D * D + (size_t)a * D : nullptr;
-        __nv_bfloat16* Dout = (live && p.st.hdiff_op)
+        __nv_bfloat16* Dout = (kDiff && live && p.st.hdiff_op)
                                   ? static_cast<__nv_bfloat16*>(p.st.hdiff_op) + ((size_t)bh * p.nb + j) * D * D + (size_t)a * D
                                   : nullptr;
 #pragma unroll
@@ -442,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
             h[x] -= hb[32 * ch + x];      // H_j - Hbar
             ss = fmaf(h[x], h[x], ss);
           }
-          if (Dout) {
+          if (kDiff && Dout) {
             // operand copy of the per-block first-order difference: s (H_j - Hbar), row a, bf16
             uint32_t pk[16];
 #pragma unroll
@@ -492,11 +495,16 @@ cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k,
   const size_t smem_a = sizeof(SmemA) + 1024, smem_b = sizeof(SmemB) + 1024;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(stats_a_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
-  if ((e = cudaFuncSetAttribute(cov_norm_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
+  if ((e = cudaFuncSetAttribute(cov_norm_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
+  if ((e = cudaFuncSetAttribute(cov_norm_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
   const int nparts = num_parts(g);
   stats_a_sm100<<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(maps, p);
   if ((e = launch_hbar_reduce(g, p.partials, nparts, p.vmax, st, stream))) return e;
-  cov_norm_sm100<<<dim3((g.nb + kBlocksPerCtaB - 1) / kBlocksPerCtaB, g.BH()), kThreads, smem_b, stream>>>(maps, p);
+  const dim3 grid_b((g.nb + kBlocksPerCtaB - 1) / kBlocksPerCtaB, g.BH());
+  if (st.hdiff_op)
+    cov_norm_sm100<true><<<grid_b, kThreads, smem_b, stream>>>(maps, p);
+  else
+    cov_norm_sm100<false><<<grid_b, kThreads, smem_b, stream>>>(maps, p);
   return cudaGetLastError();
 }
 

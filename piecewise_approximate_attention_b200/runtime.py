@@ -124,3 +124,49 @@ def choose_axis_order(pisa: "Pisa", q, k, v, perms):
         scores.append(pisa.stats.M.reshape(B * H, -1).sum(dim=1))
     best = torch.stack(scores).argmin(dim=0)
     return perms[best].contiguous(), best
+
+
+class HostPipeline:
+    """Steps whose inputs and outputs live in (pinned) host memory, with the copies overlapped:
+    the inputs of step i+1 are uploaded and the output of step i-1 is downloaded while step i
+    runs.  Two device buffer sets and three streams (upload, compute, download), ordered by
+    events; the statistics and routing buffers of `pisa` are reused by consecutive steps on the
+    compute stream.  ``submit`` only enqueues; ``synchronize`` waits for everything submitted."""
+
+    def __init__(self, pisa: "Pisa", q_like):
+        import torch
+        self.p = pisa
+        dev = pisa.device
+        self.bufs = [[torch.empty(q_like.shape, dtype=q_like.dtype, device=dev) for _ in range(4)] for _ in range(2)]
+        self.s_in, self.s_cmp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]
+        self.i = 0
+
+    def submit(self, qh, kh, vh, oh):
+        import torch
+        b = self.i % 2
+        q, k, v, o = self.bufs[b]
+        with torch.cuda.stream(self.s_in):
+            self.s_in.wait_event(self.ev_cmp[b])          # step i-2 has finished reading q, k, v
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            self.ev_in[b].record(self.s_in)
+        with torch.cuda.stream(self.s_cmp):
+            self.s_cmp.wait_event(self.ev_in[b])
+            self.s_cmp.wait_event(self.ev_out[b])         # the download of step i-2 has read o
+            self.p.precompute(q, k, v, stream=self.s_cmp)
+            self.p.route(stream=self.s_cmp)
+            self.p.attention(q, k, v, o, stream=self.s_cmp)
+            self.ev_cmp[b].record(self.s_cmp)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.ev_cmp[b])
+            oh.copy_(o, non_blocking=True)
+            self.ev_out[b].record(self.s_out)
+        self.i += 1
+
+    def synchronize(self):
+        for s in (self.s_in, self.s_cmp, self.s_out):
+            s.synchronize()

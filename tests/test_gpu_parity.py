@@ -259,3 +259,25 @@ def test_graph_replay_matches_direct_calls():
     torch.cuda.synchronize()
     assert torch.equal(o, o2)
     assert p.device_error() == (C.PISA_OK, 0)
+
+
+def test_host_pipeline_matches_direct_calls():
+    """runtime.HostPipeline (overlapped uploads, steps and downloads) gives, for every submitted
+    step, the output of a direct call on the same inputs."""
+    from piecewise_approximate_attention_b200.runtime import HostPipeline
+    w = WORKLOADS["image-dit"].with_(heads=2)
+    batches = [make_qkv(w, seed=s) for s in (0, 1, 2)]
+    B, H, L, d = batches[0][0].shape
+    p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, "cuda")
+    pipe = HostPipeline(p, batches[0][0])
+    outs = [torch.empty_like(b[0]).pin_memory() for b in batches]
+    hosts = [tuple(x.pin_memory() for x in b) for b in batches]
+    for (qh, kh, vh), oh in zip(hosts, outs):
+        pipe.submit(qh, kh, vh, oh)
+    pipe.synchronize()
+    ref = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, "cuda")
+    for (q, k, v), oh in zip(batches, outs):
+        o = ref(q.cuda(), k.cuda(), v.cuda())
+        torch.cuda.synchronize()
+        assert torch.equal(oh, o.cpu())
+    assert p.device_error() == (C.PISA_OK, 0)

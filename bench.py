@@ -35,16 +35,27 @@ def _peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def code_digest(path: str) -> str:
+    """sha256 of a CUDA source with comments and whitespace removed: it changes when the code does,
+    not when a comment does."""
+    import hashlib
+    import re
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = re.sub(r"\s+", " ", text).strip()
+    return hashlib.sha256(text.encode()).hexdigest()
+
+
 def _profiled_traffic(workload: str):
     """DRAM bytes of one attention launch from the committed ncu summary, if it was taken on the
-    attention kernel source as it is now (else None: the counters would be stale)."""
+    attention kernel code as it is now (else None: the counters would be stale)."""
     import glob
-    import hashlib
     src = os.path.join(ROOT, "piecewise_approximate_attention_b200", "csrc", "attn_sm100.cu")
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    digest = code_digest(src)
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"attn_sm100_{workload}-*.md"))):
         text = open(path).read()
-        if f"source_sha256: {sha}" in text:
+        if f"code_sha256: {digest}" in text:
             for line in text.splitlines():
                 if line.startswith("traffic_bytes_full_launch:"):
                     return int(line.split(":")[1])

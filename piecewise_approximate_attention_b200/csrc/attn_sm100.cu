@@ -16,8 +16,11 @@
 //     blocks per tile, each half masked for the query block that did not select it), then, in PISA
 //     mode, ceil(nb/128) centroid tiles (kbar_j as keys, vsum_j as values; columns of selected blocks
 //     masked).  Both kinds run through the same tcgen05 MMAs: S = Q K^T into TMEM (fp32), softmax in
-//     registers (one thread per row), P (bf16) written back over S in TMEM, O += P V with P read from
+//     registers (one thread per row), P (fp16) written back over S in TMEM, O += P V with P read from
 //     TMEM and V from shared memory (MN-major).
+//   * kF8 (PISA_BF16_FP8QK): Q, K and the centroids come as e4m3 copies and S is a kind::f8f6f4
+//     product (K = 32 per instruction); each half's raw scores are scaled by the row's q scale times
+//     the key block's (or centroid tile's) k scale.  The correction keeps the bf16 Q tile.
 //   * P enters the PV product in fp16 (11 significant bits) against an fp16 copy of the values
 //     (v / vscale, a per-head power of two, written by the pre-computation).  That precision lets
 //     the running max lag the true row max by up to 2^8 (weights up to 256), so O is rescaled in
@@ -523,7 +526,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         for (int c = 0; c < 64; ++c) slast = c == cl ? s[c] : slast;
       }
       // p = 2^(s*scale*log2e - m*scale*log2e) (masked entries are -inf and give exactly 0), two at a
-      // time with f32x2 arithmetic; P (bf16) goes over the first 32 columns of this half's S
+      // time with f32x2 arithmetic; P (fp16 pairs) goes over the first 32 columns of this half's S
       const float mb = m == -INFINITY ? 0.f : m * p.scale_log2;
       const float scl = kF8 ? p.scale_log2 * sl : p.scale_log2;
       const uint64_t sc2 = f2_pack(scl, scl), nmb2 = f2_pack(-mb, -mb);

@@ -306,10 +306,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (smooth 3D field + N(0,1) noise, seeded; stands in for Wan2.1-class video DiT activations)",
-        "config": {"workload": w.name, "batch_per_gpu": B, "heads": H, "seq_len": L, "head_dim": d,
-                   "block": w.block, "keep_k": w.keep_k, "num_blocks": p.nb, "sparsity": w.sparsity,
-                   "lambda": w.lam, "parallelism": f"weak, 1 batch element per GPU x {world}",
-                   "l2": "inputs (3 x %.0f MB) larger than L2; no flush" % (q.numel() * q.element_size() / 1e6)},
+        "config": workload_config(w, world),
         "ms_per_attention_call": round(attn_ms_max, 4),
         "ms_precompute": round(pre_ms, 4),
         "ms_route": round(route_ms, 4),
@@ -519,6 +516,15 @@ def cpu_baseline(w, heads=(0,)):
             "sample": f"{len(heads)} of {w.heads} heads of {w.name} (full pre-compute, routing and attention), fp64 numpy"}
 
 
+def workload_config(w, world: int) -> dict:
+    """The bench line's config object (the same on both arms)."""
+    tensor_mb = w.batch * w.heads * w.seq_len * w.head_dim * (2 if w.dtype == "bf16" else 4) / 1e6
+    return {"workload": w.name, "batch_per_gpu": w.batch, "heads": w.heads, "seq_len": w.seq_len,
+            "head_dim": w.head_dim, "block": w.block, "keep_k": w.keep_k, "num_blocks": w.num_blocks,
+            "sparsity": w.sparsity, "lambda": w.lam, "parallelism": f"weak, 1 batch element per GPU x {world}",
+            "l2": "inputs (3 x %.0f MB) larger than L2; no flush" % tensor_mb}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -534,7 +540,7 @@ def run_reference(args, rank, world):
     v = statistics.median(vals)
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": {"workload": w.name},
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(w, world),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
                              "sample": cb["sample"]},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

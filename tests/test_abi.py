@@ -185,3 +185,25 @@ def test_missing_library_fails_loudly(monkeypatch):
 def test_testing_hook_rejects_unknown_fault():
     assert C.lib().pisa_testing_set_attention_fault(7, 0) == C.PISA_ERR_INVALID_ARG
     assert C.lib().pisa_testing_set_attention_fault(0, 0) == C.PISA_OK
+
+
+def test_reordering_entry_points_validate_without_launch():
+    L = C.lib()
+    P = 1 << 28
+    # gather/scatter: null, misaligned, bad sizes, overlapping buffers
+    assert L.pisa_permute_rows(None, P, P, 2, 100, 256, 0, 0, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_permute_rows(P + 8, P * 2, P * 3, 2, 100, 256, 0, 0, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_permute_rows(P, P * 2, P * 3, 2, 100, 200, 0, 0, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_permute_rows(P, P * 2, P * 3, 0, 100, 256, 0, 0, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_permute_rows(P, P * 2, P * 3, 2, 0, 256, 0, 0, None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_permute_rows(P, P + 256, P * 3, 2, 100, 256, 0, 1, None) == C.PISA_ERR_INVALID_ARG
+    # axis permutation: a permutation of "thw" is required
+    out = (ctypes.c_int32 * 64)()
+    for bad in (b"thh", b"th", b"thwx", b"abc", b""):
+        assert L.pisa_axis_permutation(2, 2, 3, 0, bad, out) == C.PISA_ERR_INVALID_ARG, bad
+    assert L.pisa_axis_permutation(2, 2, 3, -1, b"thw", out) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_axis_permutation(0, 2, 3, 0, b"thw", out) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_axis_permutation(2, 2, 3, 0, b"thw", None) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_axis_permutation(2, 2, 3, 4, b"wth", out) == C.PISA_OK
+    got = list(out[:16])
+    assert sorted(got) == list(range(16)) and got[12:] == [12, 13, 14, 15]

@@ -14,8 +14,8 @@
 //   * For each block j that the tile's query blocks did not both select, the four row warps build
 //     W_j = alpha_tj q_t (one row per thread, bf16, q_t held in registers) in TMEM, and the MMA warp
 //     accumulates O += W_j (s (H_j - Hbar)), A = W_j from TMEM, B = the block's 128 x 128 bf16
-//     matrix streamed by TMA through a ring of shared-memory stages.  W has several TMEM slots, so
-//     building the next W overlaps the MMAs of the current one.  Rows whose own query block selected j get alpha = 0.
+//     matrix streamed by TMA.  W slots (TMEM) and matrix stages (shared memory) form one ring of
+//     four, so building the next W and loading the next matrices overlap the current MMAs.  Rows whose own query block selected j get alpha = 0.
 //   * The epilogue reads O from TMEM, adds the row's fp32 attention output and writes bf16.
 // Warp roles: warps 0-3 W builders + epilogue (TMEM lanes 0-127), warp 4 TMA producer, warp 5 MMA
 // issuer and TMEM owner.  Every mbarrier wait is bounded; on a timeout the CTA sets the status
@@ -33,16 +33,12 @@ constexpr int D = 128;
 constexpr int kThreads = 192;
 constexpr int kHalf = 128 * 64 * 2;        // 128 rows x 64 bf16 columns, 128B-swizzled: 16 KB
 constexpr int kTileBytes = 2 * kHalf;
-#ifndef PISA_PB_HSTAGES
-#define PISA_PB_HSTAGES 3
-#endif
-#ifndef PISA_PB_WSLOTS
-#define PISA_PB_WSLOTS 2
-#endif
-constexpr int kHS = PISA_PB_HSTAGES;       // stages of the per-block matrix ring
-constexpr int kWS = PISA_PB_WSLOTS;        // W buffers in TMEM
+// One ring of kR slots, each a W buffer in TMEM and a per-block matrix in shared memory, with one
+// "full" barrier (the producer's TMA bytes plus the 128 W builders' arrivals) and one "empty"
+// barrier (the MMAs' commit): the MMA warp waits once per block.
+constexpr int kR = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColC = 0, kColW = 128, kColO = 128 + 64 * kWS;   // C: 128 cols, W: kWS x 64, O: 128
+constexpr uint32_t kColC = 0, kColW = 128, kColO = 128 + 64 * kR;   // C: 128 cols, W: kR x 64, O: 128
 static_assert(kColO + 128 <= kTmemCols, "TMEM columns");
 constexpr int kWords = 128;                // selection bitmap words (nb <= 4096)
 constexpr int kAlphaStride = 33;
@@ -50,10 +46,10 @@ constexpr int kAlphaStride = 33;
 struct alignas(1024) Smem {
   uint8_t q[kTileBytes];
   uint8_t kb[kTileBytes];
-  uint8_t h[kHS][kTileBytes];
+  uint8_t h[kR][kTileBytes];
   float alpha[128 * kAlphaStride];          // alpha of the current 32 centroids, one row per thread
   uint64_t bar_q, bar_kfull, bar_kempty, bar_cfull, bar_cempty;
-  uint64_t bar_hfull[kHS], bar_hempty[kHS], bar_wfull[kWS], bar_wempty[kWS];
+  uint64_t bar_full[kR], bar_empty[kR];
   uint64_t bar_final, bar_drain;
   uint32_t tmem_base;
   int abort;
@@ -159,13 +155,9 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
     mbar_init(&sm.bar_kempty, 1);
     mbar_init(&sm.bar_cfull, 1);
     mbar_init(&sm.bar_cempty, 128);
-    for (int i = 0; i < kHS; ++i) {
-      mbar_init(&sm.bar_hfull[i], 1);
-      mbar_init(&sm.bar_hempty[i], 1);
-    }
-    for (int i = 0; i < kWS; ++i) {
-      mbar_init(&sm.bar_wfull[i], 128);
-      mbar_init(&sm.bar_wempty[i], 1);
+    for (int i = 0; i < kR; ++i) {
+      mbar_init(&sm.bar_full[i], 129);     // the producer's arrive.expect_tx + 128 W builders
+      mbar_init(&sm.bar_empty[i], 1);      // the MMAs' commit
     }
     mbar_init(&sm.bar_final, 1);
     mbar_init(&sm.bar_drain, 1);
@@ -220,12 +212,12 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
         for (int w = 4 * ct; w < 4 * ct + 4 && ok; ++w) {
           for (uint32_t pm = proc_word(sm, w, p.nb); pm; pm &= pm - 1) {
             const int j = 32 * w + __ffs(pm) - 1;
-            const int s = issued_h % kHS;
-            if (issued_h >= kHS && !(ok = wait_or_abort(sm, &sm.bar_hempty[s], ((issued_h / kHS) - 1) & 1, p)))
+            const int s = issued_h % kR;
+            if (issued_h >= kR && !(ok = wait_or_abort(sm, &sm.bar_empty[s], ((issued_h / kR) - 1) & 1, p)))
               break;
-            mbar_expect_tx(&sm.bar_hfull[s], kTileBytes);
-            tma_load_3d(sm.h[s], &hmap, &sm.bar_hfull[s], 0, j * D, bh);
-            tma_load_3d(sm.h[s] + kHalf, &hmap, &sm.bar_hfull[s], 64, j * D, bh);
+            mbar_expect_tx(&sm.bar_full[s], kTileBytes);
+            tma_load_3d(sm.h[s], &hmap, &sm.bar_full[s], 0, j * D, bh);
+            tma_load_3d(sm.h[s] + kHalf, &hmap, &sm.bar_full[s], 64, j * D, bh);
             ++issued_h;
           }
         }
@@ -237,8 +229,8 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
         while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
         if (issued_k > 0)
           while (!mbar_try_wait(&sm.bar_kfull, (issued_k - 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
-        for (int i = max(0, issued_h - kHS); i < issued_h; ++i)
-          while (!mbar_try_wait(&sm.bar_hfull[i % kHS], (i / kHS) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+        for (int i = max(0, issued_h - kR); i < issued_h; ++i)
+          while (!mbar_try_wait(&sm.bar_full[i % kR], (i / kR) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
       }
     }
   } else if (warp == 5) {
@@ -263,17 +255,15 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
         mma_commit(&sm.bar_cfull);
         for (int w = 4 * ct; w < 4 * ct + 4 && ok; ++w) {
           for (uint32_t pm = proc_word(sm, w, p.nb); pm; pm &= pm - 1) {
-            const int slot = n % kWS, s = n % kHS;
-            if (!(ok = wait_or_abort(sm, &sm.bar_wfull[slot], (n / kWS) & 1, p))) break;
-            if (!(ok = wait_or_abort(sm, &sm.bar_hfull[s], (n / kHS) & 1, p))) break;
+            const int slot = n % kR, s = slot;
+            if (!(ok = wait_or_abort(sm, &sm.bar_full[slot], (n / kR) & 1, p))) break;
             tc_fence_after();
             const uint64_t hd = smem_desc_sw128(smem_u32(sm.h[s]), kHalf, 1024);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ts(tmem + kColO, tmem + kColW + 64 * slot + 8 * kk, hd + (uint64_t)(kk * 2048 >> 4), idesc_h,
                      (n > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&sm.bar_wempty[slot]);
-            mma_commit(&sm.bar_hempty[s]);
+            mma_commit(&sm.bar_empty[slot]);
             ++n;
           }
         }
@@ -330,9 +320,9 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
         for (int x = 0; x < 32; ++x)
           arow[x] = ((am >> x) & 1u) ? ex2(fmaf(c[x], p.scale_log2, -rs.x)) * rs.y : 0.f;
         for (uint32_t mm = pm; mm; mm &= mm - 1) {
-          const int x = __ffs(mm) - 1, slot = n % kWS;
-          if (n >= kWS) {
-            ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_wempty[slot], ((n / kWS) - 1) & 1, p));
+          const int x = __ffs(mm) - 1, slot = n % kR;
+          if (n >= kR) {
+            ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_empty[slot], ((n / kR) - 1) & 1, p));
             if (!ok) break;
             tc_fence_after();
           }
@@ -345,7 +335,7 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
           tmem_st32(trow + kColW + 64 * slot + 32, reinterpret_cast<const float*>(wv + 32));
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&sm.bar_wfull[slot]);
+          mbar_arrive(&sm.bar_full[slot]);
           ++n;
         }
       }

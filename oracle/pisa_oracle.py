@@ -362,8 +362,9 @@ def pisa_reordered(q, k, v, perm, block: int, keep_k: int, lam: float, scale: fl
 
 
 # --------------------------------------------------------------------------------------------
-# e4m3 logits for the exact stage (SURVEY's next row on low-bit attention, after PAROAttention's
-# INT8/INT4 remark in its abstract; the pages give no FP8 recipe, so this is a reading).  The
+# e4m3 logits for the exact stage (low-bit attention in the spirit of the INT8/INT4 attention that
+# "PAROAttention: Pattern-Aware ReOrdering ..." mentions in its abstract; no page gives an FP8
+# recipe, so this is a reading).  The
 # exact and zeroth-order logits use e4m3 copies of q (one scale per row), k (one scale per key
 # block) and kbar (one scale per tile of 128 centroids); the scale of a group is max|x| / 448 and
 # the code of x is e4m3(x / scale), both decided in float32.  Routing, the values and the

@@ -138,6 +138,10 @@ EDGE = [
     ("fp32", (2, 5, 5), 0, 64, 0, 0.5, C.PISA_MODE_PISA),
     ("fp32", (1, 19, 20), 9, 128, 2, 0.5, C.PISA_MODE_PER_BLOCK),
     ("fp32", (2, 5, 5), 0, 64, 0, 0.5, C.PISA_MODE_PER_BLOCK),
+    # a single token: one block of one row (the centroid is the token, every H_j is 0)
+    ("bf16", (1, 1, 1), 0, 64, 0, 0.5, C.PISA_MODE_PISA),
+    ("bf16", (1, 1, 1), 0, 128, 1, 0.5, C.PISA_MODE_PISA),
+    ("fp32", (1, 1, 1), 0, 64, 0, 0.5, C.PISA_MODE_PISA),
 ]
 # the bf16 tensor-core path is built for head_dim 128 only; fp32 runs both head sizes
 EDGE_CASES = [(c, hd) for c in EDGE for hd in ((64, 128) if c[0] == "fp32" else (128,))]
@@ -281,3 +285,21 @@ def test_host_pipeline_matches_direct_calls():
         torch.cuda.synchronize()
         assert torch.equal(oh, o.cpu())
     assert p.device_error() == (C.PISA_OK, 0)
+
+
+
+def test_maximum_block_count():
+    """nb = 4096, the largest supported: 262144 tokens in 64-token blocks (the router then works on
+    8 query blocks per CTA and the selection bitmaps are full), sampled query blocks."""
+    w = Workload("max-nb", 1, 1, (64, 64, 64), 0, 128, 64, 1.0 - 64 / 4096, 0.5, "bf16", seed=21)
+    assert w.num_blocks == 4096 and w.keep_k == 64
+    q, k, v = make_qkv(w)
+    p, o, scores, qkv = _run(w, q, k, v)
+    qblocks = [0, 1, 2047, 4094, 4095]
+    ref = O.pisa(_np(q), _np(k), _np(v), w.block, w.keep_k, w.lam, qblocks=qblocks)
+    _check_stats(p, ref, 0, 0, 0, 1e-4)
+    bad, ties = compare_selection(p.sel[0, 0].cpu().numpy(), ref["sel"][0, 0], ref["r"][0, 0], w.keep_k)
+    assert not bad, f"selection rows differ beyond ties: {bad[:10]}"
+    o2 = _attention_with(p, qkv, ref["sel"][0, 0], 0, 0, o)
+    rows = rows_of_blocks(w.seq_len, w.block, qblocks)
+    assert_output(_np(o2[0, 0])[rows], ref["o"][0, 0][rows], "bf16", what="nb 4096, oracle selection")

@@ -49,3 +49,31 @@ def test_wait_timeout_is_reported_and_context_survives():
     assert not bad
     keep = ~rows_of_blocks(w.seq_len, w.block, ties)
     assert_output(o2[0, 0].double().cpu().numpy()[keep], ref["o"][0, 0][keep], "bf16", what="after timeout")
+
+
+@pytest.mark.parametrize("dtype,mode", [("bf16_fp8qk", C.PISA_MODE_PISA), ("bf16", C.PISA_MODE_PER_BLOCK)])
+def test_wait_timeout_in_other_paths(dtype, mode):
+    """The same bounded wait in the e4m3-logit instantiation, and in the per-block mode, where the
+    second kernel runs after the timed-out one on whatever the workspace holds (it waits only on
+    its own copies and MMAs, so it ends too); the status is reported and the context survives."""
+    w = Workload("fault", 1, 1, (2, 16, 16), 0, 128, 64, 0.5, 0.5, "bf16", seed=3)
+    q, k, v = make_qkv(w)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    p = Pisa(1, 1, w.seq_len, 128, w.block, w.keep_k, w.lam, dtype, 1.0, "cuda", mode)
+    p.precompute(qd, kd, vd)
+    p.route()
+    torch.cuda.synchronize()
+    assert p.device_error() == (C.PISA_OK, 0)
+    o = torch.zeros_like(qd)
+    assert C.lib().pisa_testing_set_attention_fault(SKIP_Q_LOAD, WAIT_NS) == C.PISA_OK
+    try:
+        p.attention(qd, kd, vd, o)
+        torch.cuda.synchronize()
+    finally:
+        assert C.lib().pisa_testing_set_attention_fault(0, 0) == C.PISA_OK
+    assert p.device_error() == (C.PISA_ERR_DEVICE_TIMEOUT, C.PISA_DEVERR_WAIT_TIMEOUT)
+    o2 = torch.empty_like(qd)
+    p.attention(qd, kd, vd, o2)
+    torch.cuda.synchronize()
+    assert p.device_error() == (C.PISA_OK, 0)
+    assert torch.isfinite(o2).all()

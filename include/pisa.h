@@ -210,7 +210,8 @@ PISA_API pisa_status pisa_permute_rows(const void* src, void* dst, const int32_t
                                        int32_t seq_len, int32_t row_bytes, int32_t perm_per_head, int32_t inverse,
                                        pisa_stream_t stream);
 
-/* Host-only helper (perm_host is a HOST buffer of frames*height*width + extra_tokens int32): the
+/* Host-only helper (perm_host is a HOST buffer of `capacity` int32, at least
+ * frames*height*width + extra_tokens; a smaller capacity returns PISA_ERR_INVALID_ARG): the
  * permutation that lists the tokens of a frames x height x width grid, stored in raster order
  * (t slowest, then h, then w), in the axis order `order` — a NUL-terminated string of the three
  * distinct characters 't', 'h', 'w', slowest axis first ("thw" is the identity, "hwt" makes the
@@ -218,7 +219,7 @@ PISA_API pisa_status pisa_permute_rows(const void* src, void* dst, const int32_t
  * extra_tokens rows after the grid (e.g. text tokens) keep their place at the end.  Enqueues
  * nothing; PISA_ERR_INVALID_ARG for a bad order or size. */
 PISA_API pisa_status pisa_axis_permutation(int32_t frames, int32_t height, int32_t width, int32_t extra_tokens,
-                                           const char* order, int32_t* perm_host);
+                                           const char* order, int32_t* perm_host, int64_t capacity);
 
 /* Synchronises `stream`, copies the device status word out of ws into *code (0 = clean; otherwise
  * a PISA_DEVERR_* value below) and clears it.  Returns PISA_ERR_DEVICE_TIMEOUT when a bounded wait

@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
             "pisa_precompute_noalloc": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp]),
             "pisa_testing_set_attention_fault": (i32, [i32, ctypes.c_uint64]),
             "pisa_permute_rows": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp]),
-            "pisa_axis_permutation": (i32, [i32, i32, i32, i32, ctypes.c_char_p, P(i32)]),
+            "pisa_axis_permutation": (i32, [i32, i32, i32, i32, ctypes.c_char_p, P(i32), ctypes.c_int64]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -236,7 +236,8 @@ def pisa_axis_permutation(grid, order: str, extra_tokens: int = 0):
     T, Hg, W = grid
     out = np.empty(T * Hg * W + extra_tokens, dtype=np.int32)
     _check(lib().pisa_axis_permutation(T, Hg, W, extra_tokens, order.encode(),
-                                       out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))), "pisa_axis_permutation")
+                                       out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), out.size),
+           "pisa_axis_permutation")
     return out
 
 

@@ -98,7 +98,7 @@ using namespace pisa;
 
 extern "C" {
 
-int32_t pisa_abi_version(void) { return 4; }
+int32_t pisa_abi_version(void) { return 5; }
 
 int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
   if (seq_len < 1 || block < 1) return -1;
@@ -269,9 +269,10 @@ pisa_status pisa_permute_rows(const void* src, void* dst, const int32_t* perm, i
 }
 
 pisa_status pisa_axis_permutation(int32_t frames, int32_t height, int32_t width, int32_t extra_tokens,
-                                  const char* order, int32_t* perm_host) {
+                                  const char* order, int32_t* perm_host, int64_t capacity) {
   if (frames < 1 || height < 1 || width < 1 || extra_tokens < 0 || !order || !perm_host) return PISA_ERR_INVALID_ARG;
-  if ((long long)frames * height * width + extra_tokens > 0x7fffffffLL) return PISA_ERR_INVALID_ARG;
+  const long long total = (long long)frames * height * width + extra_tokens;
+  if (total > 0x7fffffffLL || capacity < total) return PISA_ERR_INVALID_ARG;
   // order: the three axes t, h, w, slowest first
   int axis[3], seen = 0;
   for (int i = 0; i < 3; ++i) {

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_blocks():
-    assert C.lib().pisa_abi_version() == 4
+    assert C.lib().pisa_abi_version() == 5
     assert C.pisa_num_blocks(32760, 64) == 512
     assert C.pisa_num_blocks(75600, 128) == 591
     assert C.pisa_num_blocks(1, 64) == 1
@@ -200,10 +200,11 @@ def test_reordering_entry_points_validate_without_launch():
     # axis permutation: a permutation of "thw" is required
     out = (ctypes.c_int32 * 64)()
     for bad in (b"thh", b"th", b"thwx", b"abc", b""):
-        assert L.pisa_axis_permutation(2, 2, 3, 0, bad, out) == C.PISA_ERR_INVALID_ARG, bad
-    assert L.pisa_axis_permutation(2, 2, 3, -1, b"thw", out) == C.PISA_ERR_INVALID_ARG
-    assert L.pisa_axis_permutation(0, 2, 3, 0, b"thw", out) == C.PISA_ERR_INVALID_ARG
-    assert L.pisa_axis_permutation(2, 2, 3, 0, b"thw", None) == C.PISA_ERR_INVALID_ARG
-    assert L.pisa_axis_permutation(2, 2, 3, 4, b"wth", out) == C.PISA_OK
+        assert L.pisa_axis_permutation(2, 2, 3, 0, bad, out, 64) == C.PISA_ERR_INVALID_ARG, bad
+    assert L.pisa_axis_permutation(2, 2, 3, -1, b"thw", out, 64) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_axis_permutation(0, 2, 3, 0, b"thw", out, 64) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_axis_permutation(2, 2, 3, 0, b"thw", None, 64) == C.PISA_ERR_INVALID_ARG
+    assert L.pisa_axis_permutation(2, 2, 3, 4, b"wth", out, 15) == C.PISA_ERR_INVALID_ARG   # needs 16
+    assert L.pisa_axis_permutation(2, 2, 3, 4, b"wth", out, 16) == C.PISA_OK
     got = list(out[:16])
     assert sorted(got) == list(range(16)) and got[12:] == [12, 13, 14, 15]

@@ -180,78 +180,72 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
   }
 }
 
-// Query-block pairing for 128-row tiles when block == 64: a greedy pass in index order pairs
-// each unpaired query block i with the unpaired block p in (i, i + kWin] whose selection shares
-// the most key blocks with S_i (ties to the nearer p).  Blocks left without a partner go last.
-// The attention result does not depend on the order; only the union of S_i and S_p, which one
-// tile iterates over, does.  One CTA per head; bitmaps of the selections live in shared memory.
-constexpr int kWin = 128;
-constexpr int kChunk = 64;
+// Query-block pairing for 128-row tiles when block == 64.  The query blocks are cut into segments
+// of kSeg consecutive blocks, one CTA each; inside a segment a greedy pass in index order pairs each
+// unpaired block i with the unpaired block p of the same segment (p > i) whose selection shares the
+// most key blocks with S_i (ties to the nearer p).  Pairs fill the segment's range of the order
+// first, blocks left without a partner follow, so no tile straddles two segments (a full segment
+// holds an even count).  The attention result does not depend on the order; only the union of S_i
+// and S_p, which one tile iterates over, does.  Bitmaps of the selections live in shared memory.
+constexpr int kSeg = 128;
 
 __global__ void __launch_bounds__(kThreads) pair_kernel(const int32_t* __restrict__ sel, int nb, int keep_k,
                                                         int32_t* __restrict__ order) {
   extern __shared__ uint32_t psm[];
   const int nwords = (nb + 31) / 32;
-  uint32_t* bits = psm;                                            // [kChunk + kWin][nwords]
-  uint16_t* ov = reinterpret_cast<uint16_t*>(bits + (kChunk + kWin) * nwords);  // [kChunk][kWin]
-  uint32_t* used = reinterpret_cast<uint32_t*>(ov + kChunk * kWin);             // [nwords]
-  int32_t* singles = reinterpret_cast<int32_t*>(used + nwords);                 // [nb]
+  uint32_t* bits = psm;                                                  // [kSeg][nwords]
+  uint16_t* ov = reinterpret_cast<uint16_t*>(bits + kSeg * nwords);     // [kSeg][kSeg], a < b used
+  int32_t* singles = reinterpret_cast<int32_t*>(ov + kSeg * kSeg);      // [kSeg]
+  __shared__ uint32_t used[kSeg / 32];
   __shared__ int npos, nsingle;
-  const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int32_t* S = sel + (size_t)bh * nb * keep_k;
-  int32_t* out = order + (size_t)bh * nb;
-  for (int w = threadIdx.x; w < nwords; w += kThreads) used[w] = 0u;
+  const int bh = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s0 = blockIdx.x * kSeg, n = min(kSeg, nb - s0);
+  const int32_t* S = sel + ((size_t)bh * nb + s0) * keep_k;
+  int32_t* out = order + (size_t)bh * nb + s0;
+  for (int e = threadIdx.x; e < kSeg * nwords; e += kThreads) bits[e] = 0u;
+  if (threadIdx.x < kSeg / 32) used[threadIdx.x] = 0u;
   if (threadIdx.x == 0) { npos = 0; nsingle = 0; }
-  for (int c0 = 0; c0 < nb; c0 += kChunk) {
-    const int nrows = min(nb - c0, kChunk + kWin);
-    __syncthreads();
-    for (int e = threadIdx.x; e < (kChunk + kWin) * nwords; e += kThreads) bits[e] = 0u;
-    __syncthreads();
-    for (int e = threadIdx.x; e < nrows * keep_k; e += kThreads) {
-      const int r = e / keep_k;
-      const int j = S[(size_t)(c0 + r) * keep_k + e % keep_k];
-      if (j >= 0 && j < nb) atomicOr(&bits[r * nwords + (j >> 5)], 1u << (j & 31));
+  __syncthreads();
+  for (int e = threadIdx.x; e < n * keep_k; e += kThreads) {
+    const int r = e / keep_k;
+    const int j = S[(size_t)r * keep_k + e % keep_k];
+    if (j >= 0 && j < nb) atomicOr(&bits[r * nwords + (j >> 5)], 1u << (j & 31));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kSeg * kSeg; e += kThreads) {
+    const int x = e / kSeg, y = e % kSeg;
+    int cnt = 0;
+    if (x < y && y < n) {
+      const uint32_t* bx = bits + x * nwords;
+      const uint32_t* by = bits + y * nwords;
+      for (int w = 0; w < nwords; ++w) cnt += __popc(bx[w] & by[w]);
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < kChunk * kWin; e += kThreads) {
-      const int a = e / kWin, dl = e % kWin + 1;
-      int cnt = 0;
-      if (a + dl < nrows) {
-        const uint32_t* x = bits + a * nwords;
-        const uint32_t* y = bits + (a + dl) * nwords;
-        for (int w = 0; w < nwords; ++w) cnt += __popc(x[w] & y[w]);
+    ov[e] = (uint16_t)cnt;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    for (int a = 0; a < n; ++a) {
+      if ((used[a >> 5] >> (a & 31)) & 1u) continue;
+      // best partner packed as ((overlap + 1) << 8) | (255 - distance): one warp max picks it (0 = none)
+      uint32_t key = 0u;
+      for (int b = a + 1 + lane; b < n; b += 32) {
+        if (!((used[b >> 5] >> (b & 31)) & 1u))
+          key = max(key, ((uint32_t)(ov[a * kSeg + b] + 1) << 8) | (uint32_t)(255 - (b - a)));
       }
-      ov[e] = (uint16_t)cnt;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      for (int a = 0; a < kChunk && c0 + a < nb; ++a) {
-        const int i = c0 + a;
-        if ((used[i >> 5] >> (i & 31)) & 1u) continue;
-        // best partner: most shared key blocks, ties to the nearer one; packed as
-        // ((overlap + 1) << 8) | (255 - distance) so one warp max reduction picks it (0 = none)
-        uint32_t key = 0u;
-        for (int dl = lane + 1; dl <= kWin; dl += 32) {
-          const int p = i + dl;
-          if (p < nb && !((used[p >> 5] >> (p & 31)) & 1u))
-            key = max(key, ((uint32_t)(ov[a * kWin + dl - 1] + 1) << 8) | (uint32_t)(255 - dl));
+      key = __reduce_max_sync(0xffffffffu, key);
+      if (lane == 0) {
+        used[a >> 5] |= 1u << (a & 31);
+        if (key) {
+          const int b = a + 255 - (int)(key & 255u);
+          used[b >> 5] |= 1u << (b & 31);
+          out[npos] = s0 + a;
+          out[npos + 1] = s0 + b;
+          npos += 2;
+        } else {
+          singles[nsingle++] = s0 + a;
         }
-        key = __reduce_max_sync(0xffffffffu, key);
-        const int best = key ? 255 - (int)(key & 255u) : -1;
-        if (lane == 0) {
-          used[i >> 5] |= 1u << (i & 31);
-          if (best > 0) {
-            const int p = i + best;
-            used[p >> 5] |= 1u << (p & 31);
-            out[npos] = i;
-            out[npos + 1] = p;
-            npos += 2;
-          } else {
-            singles[nsingle++] = i;
-          }
-        }
-        __syncwarp();
       }
+      __syncwarp();
     }
   }
   __syncthreads();
@@ -293,10 +287,9 @@ cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float 
   if (order) {
     if (g.block == 64 && keep_k > 0 && g.nb > 2) {
       const int nwords = (g.nb + 31) / 32;
-      const size_t psmem = (size_t)(kChunk + kWin) * nwords * 4 + (size_t)kChunk * kWin * 2 + (size_t)nwords * 4 +
-                           (size_t)g.nb * 4;
+      const size_t psmem = (size_t)kSeg * nwords * 4 + (size_t)kSeg * kSeg * 2 + (size_t)kSeg * 4;
       if ((e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem))) return e;
-      pair_kernel<<<g.BH(), kThreads, psmem, stream>>>(sel, g.nb, keep_k, order);
+      pair_kernel<<<dim3((g.nb + kSeg - 1) / kSeg, g.BH()), kThreads, psmem, stream>>>(sel, g.nb, keep_k, order);
     } else {
       identity_order<<<dim3((g.nb + 255) / 256, g.BH()), 256, 0, stream>>>(g.nb, order);
     }

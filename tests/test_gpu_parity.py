@@ -201,13 +201,18 @@ def test_value_operand_copy_and_large_values():
         assert_output(_np(o2[0, h])[keep], ref["o"][0, h][keep], "bf16", what=f"large values head {h}")
 
 
-def test_order_is_a_permutation():
-    w = WORKLOADS["video-dit-small"].with_(heads=2)
+@pytest.mark.parametrize("grid", [(21, 30, 52), (2, 59, 109)])
+def test_order_is_a_permutation(grid):
+    # 512 query blocks (four pairing segments of 128) and 201 (a ragged last segment of 73)
+    w = WORKLOADS["video-dit-small"].with_(heads=2, grid=grid)
     q, k, v = make_qkv(w)
     p, _, _, _ = _run(w, q, k, v)
     od = p.order.cpu().numpy()
     for h in range(2):
         assert sorted(od[0, h].tolist()) == list(range(w.num_blocks))
+        # pairs never straddle a segment: the two blocks of each 128-row tile lie in one segment
+        tiles = od[0, h][: w.num_blocks // 2 * 2].reshape(-1, 2) // 128
+        assert np.array_equal(tiles[:, 0], tiles[:, 1])
 
 
 def test_deterministic():

@@ -470,15 +470,9 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
           }
         }
       }
-      ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_sfull[hh], t & 1, p));
-      if (!ok) break;
-      tc_fence_after();
-      const float sl = kF8 ? qsc * (hh ? ksc1 : ksc0) : 1.f;   // raw MMA score -> logit
       const bool centroid = kt.kind == 1;
-      float s[64];
-      tmem_ld32(trow + kColS + 64 * hh, s);
-      tmem_ld32(trow + kColS + 64 * hh + 32, s + 32);
-      // validity of this half's 64 columns, 32 per word
+      // validity of this half's 64 columns for this row's query block, 32 per word (warp-uniform:
+      // a warp's rows belong to one query block)
       uint32_t vm0, vm1;
       if (!centroid) {
         const int jh = pair ? (hh ? kt.j1 : kt.j0) : kt.j0;
@@ -492,6 +486,27 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
         vm0 = (r0 >= 32 ? FULL : (r0 > 0 ? ((1u << r0) - 1u) : 0u)) & ~(w0 < kWords ? bits[w0] : 0u);
         vm1 = (r1 >= 32 ? FULL : (r1 > 0 ? ((1u << r1) - 1u) : 0u)) & ~(w0 + 1 < kWords ? bits[w0 + 1] : 0u);
       }
+      ok = __all_sync(FULL, wait_or_abort(sm, &sm.bar_sfull[hh], t & 1, p));
+      if (!ok) break;
+      tc_fence_after();
+      if (__all_sync(FULL, (vm0 | vm1) == 0u)) {
+        // Every column masked for this warp's rows (in a paired tile, a key block that only the other
+        // query block selected): all weights are exactly 0 and m, l, A stay as they are, so the scores
+        // are not read and only P = 0 is written for the PV product.
+        uint32_t zero[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) zero[x] = 0u;
+        tmem_st16(trow + kColS + 64 * hh, zero);
+        tmem_st16(trow + kColS + 64 * hh + 16, zero);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sm.bar_pfull[hh]);
+        continue;
+      }
+      const float sl = kF8 ? qsc * (hh ? ksc1 : ksc0) : 1.f;   // raw MMA score -> logit
+      float s[64];
+      tmem_ld32(trow + kColS + 64 * hh, s);
+      tmem_ld32(trow + kColS + 64 * hh + 32, s + 32);
       tmem_ld_wait();
       if (vm0 != FULL) {
 #pragma unroll

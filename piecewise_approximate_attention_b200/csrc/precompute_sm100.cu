@@ -107,7 +107,7 @@ struct alignas(1024) SmemA {
   uint8_t q[2][kTile];
   uint8_t k[2][kTile];
   uint8_t v[2][kTile];
-  float red[3][8][128];
+  float red[3][4][128];
   float ck[2][128], cv[2][128];
   uint64_t full[2], empty[2], acc_done;
   uint32_t tmem_base;
@@ -205,17 +205,30 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
         colsum8(sm.q[s], cc, rg, r0, r0 + cnt, aq);
         colsum8(sm.k[s], cc, rg, r0, r0 + cnt, ak);
         colsum8(sm.v[s], cc, rg, r0, r0 + cnt, av, &vabs);
+        // lanes l and l ^ 16 hold the same 8 columns for row groups 2w and 2w + 1: add them in
+        // registers, then one row of partial sums per warp goes through shared memory
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          sm.red[0][rg][cc * 8 + x] = aq[x];
-          sm.red[1][rg][cc * 8 + x] = ak[x];
-          sm.red[2][rg][cc * 8 + x] = av[x];
+          aq[x] += __shfl_xor_sync(0xffffffffu, aq[x], 16);
+          ak[x] += __shfl_xor_sync(0xffffffffu, ak[x], 16);
+          av[x] += __shfl_xor_sync(0xffffffffu, av[x], 16);
+        }
+        if (lane < 16) {
+          float4* dq = reinterpret_cast<float4*>(&sm.red[0][warp][cc * 8]);
+          float4* dk = reinterpret_cast<float4*>(&sm.red[1][warp][cc * 8]);
+          float4* dv = reinterpret_cast<float4*>(&sm.red[2][warp][cc * 8]);
+          dq[0] = make_float4(aq[0], aq[1], aq[2], aq[3]);
+          dq[1] = make_float4(aq[4], aq[5], aq[6], aq[7]);
+          dk[0] = make_float4(ak[0], ak[1], ak[2], ak[3]);
+          dk[1] = make_float4(ak[4], ak[5], ak[6], ak[7]);
+          dv[0] = make_float4(av[0], av[1], av[2], av[3]);
+          dv[1] = make_float4(av[4], av[5], av[6], av[7]);
         }
         bar_epi();
         const int c = tid;
         float sq = 0.f, sk = 0.f, sv = 0.f;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
+        for (int g = 0; g < 4; ++g) {
           sq += sm.red[0][g][c];
           sk += sm.red[1][g][c];
           sv += sm.red[2][g][c];
@@ -283,7 +296,8 @@ constexpr int kBlocksPerCtaB = 16;
 struct alignas(1024) SmemB {
   uint8_t k[kStagesB][kTile];
   uint8_t v[kStagesB][kTile];
-  float vs[2][2][128];
+  float kbp[kBlocksPerCtaB][128];   // this CTA's centroids kbar_j and value sums vsum_j
+  float vsp[kBlocksPerCtaB][128];
   float red[2][4];
   uint64_t full[kStagesB], empty[kStagesB], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
@@ -379,6 +393,24 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
     const float vinv = 1.f / p.st.vscale[bh];
     __half* vop = reinterpret_cast<__half*>(p.st.v_op) + (size_t)bh * p.L * D;
     __half* vsop = reinterpret_cast<__half*>(p.st.vsum_op);
+    {
+      // column a of every block's kbar and vsum, all loads issued before the first use; the fp16
+      // operand copy vsum / vscale is written here too
+      float kv[kBlocksPerCtaB], vv[kBlocksPerCtaB];
+#pragma unroll
+      for (int jj = 0; jj < kBlocksPerCtaB; ++jj) {
+        const size_t so = ((size_t)bh * p.nb + min(jb0 + jj, jb1 - 1)) * D + a;
+        kv[jj] = p.st.kbar[so];
+        vv[jj] = p.st.vsum[so];
+      }
+#pragma unroll
+      for (int jj = 0; jj < kBlocksPerCtaB; ++jj) {
+        sm.kbp[jj][a] = kv[jj];
+        sm.vsp[jj][a] = vv[jj];
+        if (jb0 + jj < jb1) vsop[((size_t)bh * p.nb + jb0 + jj) * D + a] = __float2half_rn(vv[jj] * vinv);
+      }
+      bar_epi();
+    }
     float hb[D];
     const float* hbar = p.st.hbar + (size_t)bh * D * D + (size_t)a * D;
 #pragma unroll
@@ -418,11 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
       for (int b = 0; b < bpt; ++b) {
         const int j = jb0 + t * bpt + b;
         const bool live = j < jb1;
-        const size_t so = ((size_t)bh * p.nb + (live ? j : 0)) * D;
-        sm.vs[buf][b][a] = live ? p.st.vsum[so + a] : 0.f;
-        if (live) vsop[so + a] = __float2half_rn(sm.vs[buf][b][a] * vinv);
-        const float kb = live ? p.st.kbar[so + a] : 0.f;
-        bar_epi();
+        const float* vsj = sm.vsp[live ? j - jb0 : 0];
+        const float kb = live ? sm.kbp[j - jb0][a] : 0.f;   // 0: a missing block's H stays unused
+        const int rb = (t * bpt + b) & 1;                    // red[] alternates between blocks
         float ss = 0.f;
         float* Hout = (live && p.st.H) ? p.st.H + ((size_t)bh * p.nb + j) * D * D + (size_t)a * D : nullptr;
         __nv_bfloat16* Dout = (kDiff && live && p.st.hdiff_op)
@@ -434,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
           tmem_ld32(trow + (uint32_t)(buf * 256 + b * 128 + 32 * ch), h);
           tmem_ld_wait();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) h[x] = fmaf(-kb, sm.vs[buf][b][32 * ch + x], h[x]);
+          for (int x = 0; x < 32; ++x) h[x] = fmaf(-kb, vsj[32 * ch + x], h[x]);
           if (Hout) {
 #pragma unroll
             for (int x = 0; x < 32; x += 4)
@@ -456,9 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
           }
         }
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if (lane == 0) sm.red[b][warp] = ss;
+        if (lane == 0) sm.red[rb][warp] = ss;
         bar_epi();
-        if (a == 0 && live) p.st.M[(size_t)bh * p.nb + j] = sqrtf(sm.red[b][0] + sm.red[b][1] + sm.red[b][2] + sm.red[b][3]);
+        if (a == 0 && live) p.st.M[(size_t)bh * p.nb + j] = sqrtf(sm.red[rb][0] + sm.red[rb][1] + sm.red[rb][2] + sm.red[rb][3]);
       }
       tc_fence_before();
       mbar_arrive(&sm.acc_empty[buf]);

@@ -97,7 +97,7 @@ template <int kRows>
 constexpr int tile_j() { return 4 * kThreads / kRows; }
 
 template <int D, int kRows>
-__global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
+__global__ void __launch_bounds__(kThreads, 2) route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
                                                          const float* __restrict__ M, int L, int block, int nb,
                                                          float scale, int keep_k, float lam,
                                                          int32_t* __restrict__ sel, float* __restrict__ scores) {
@@ -108,32 +108,53 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
   float* r = ks + kTileJ * (D + 4);                        // [kRows][nb]
   uint32_t* hist = reinterpret_cast<uint32_t*>(r + kRows * nb);   // [kWarps][256]
   float* red = reinterpret_cast<float*>(hist + kWarps * 256);     // [kWarps]
+  float* Ms = red + kWarps;                                       // [nb]: M_j of this head
   const int bh = blockIdx.y, i0 = blockIdx.x * kRows;
   const int rows = min(kRows, nb - i0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* Mh = M + (size_t)bh * nb;
 
-  for (int idx = threadIdx.x; idx < kRows * D; idx += kThreads) {
-    const int ri = idx / D;
+  static_assert(kRows * D % kThreads == 0, "query rows per thread");
+#pragma unroll
+  for (int x = 0; x < kRows * D / kThreads; ++x) {
+    const int idx = threadIdx.x + x * kThreads, ri = idx / D;
     qs[idx] = ri < rows ? scale * qbar[((size_t)bh * nb + i0 + ri) * D + idx % D] : 0.f;
   }
-  // sum_l M_l in a fixed order
+  // M_j kept in shared memory for the rows below; sum_l M_l in a fixed order
   float msum = 0.f;
-  for (int j = threadIdx.x; j < nb; j += kThreads) msum += Mh[j];
+#pragma unroll 4
+  for (int j = threadIdx.x; j < nb; j += kThreads) {
+    const float mv = Mh[j];
+    Ms[j] = mv;
+    msum += mv;
+  }
   msum = warp_sum(msum);
   if (lane == 0) red[warp] = msum;
 
   const int jj = threadIdx.x % kTileJ, g = threadIdx.x / kTileJ;   // centroid column, query group
   const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nb * D);
+  // the next k̄ tile is loaded into registers while the current one is used
+  constexpr int kLoads = kTileJ * (D / 4) / kThreads;
+  static_assert(kLoads * kThreads == kTileJ * (D / 4), "tile loads per thread");
+  float4 nxt[kLoads];
+  auto load_tile = [&](int j0) {
+#pragma unroll
+    for (int x = 0; x < kLoads; ++x) {
+      const int idx = threadIdx.x + x * kThreads, jr = idx / (D / 4), a4 = idx % (D / 4);
+      nxt[x] = j0 + jr < nb ? kb4[(size_t)(j0 + jr) * (D / 4) + a4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  load_tile(0);
   for (int j0 = 0; j0 < nb; j0 += kTileJ) {
     const int nj = min(kTileJ, nb - j0);
     __syncthreads();
-    for (int idx = threadIdx.x; idx < kTileJ * (D / 4); idx += kThreads) {
-      const int jr = idx / (D / 4), a4 = idx % (D / 4);
-      const float4 v = jr < nj ? kb4[(size_t)(j0 + jr) * (D / 4) + a4] : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(ks + jr * (D + 4) + 4 * a4) = v;
+#pragma unroll
+    for (int x = 0; x < kLoads; ++x) {
+      const int idx = threadIdx.x + x * kThreads, jr = idx / (D / 4), a4 = idx % (D / 4);
+      *reinterpret_cast<float4*>(ks + jr * (D + 4) + 4 * a4) = nxt[x];
     }
     __syncthreads();
+    if (j0 + kTileJ < nb) load_tile(j0 + kTileJ);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const float* kr = ks + jj * (D + 4);
 #pragma unroll 8
@@ -171,7 +192,7 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
     const float inv = 1.f / den;
     const size_t row = (size_t)bh * nb + i0 + ri;
     for (int j = lane; j < nb; j += 32) {
-      const float val = rr[j] * inv + minv * Mh[j];
+      const float val = rr[j] * inv + minv * Ms[j];
       rr[j] = val;
       if (scores) scores[row * nb + j] = val;
     }
@@ -188,68 +209,99 @@ __global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict
 // holds an even count).  The attention result does not depend on the order; only the union of S_i
 // and S_p, which one tile iterates over, does.  Bitmaps of the selections live in shared memory.
 constexpr int kSeg = 128;
+static_assert(kSeg == 128, "the pairing pass keeps a segment's set of paired blocks in four 32-bit words");
+
+// Bit b of a 128-bit set held as four words in registers (the same value in every lane).
+__device__ __forceinline__ bool bit128(uint32_t u0, uint32_t u1, uint32_t u2, uint32_t u3, int b) {
+  const int w = b >> 5;
+  const uint32_t x = w == 0 ? u0 : (w == 1 ? u1 : (w == 2 ? u2 : u3));
+  return (x >> (b & 31)) & 1u;
+}
 
 __global__ void __launch_bounds__(kThreads) pair_kernel(const int32_t* __restrict__ sel, int nb, int keep_k,
                                                         int32_t* __restrict__ order) {
   extern __shared__ uint32_t psm[];
   const int nwords = (nb + 31) / 32;
-  uint32_t* bits = psm;                                                  // [kSeg][nwords]
+  // word-major bitmaps: word w of block y at bits[w * kSeg + y], so a warp reading 32 consecutive
+  // blocks' words touches 32 banks
+  uint32_t* bits = psm;                                                  // [nwords][kSeg]
   uint16_t* ov = reinterpret_cast<uint16_t*>(bits + kSeg * nwords);     // [kSeg][kSeg], a < b used
   int32_t* singles = reinterpret_cast<int32_t*>(ov + kSeg * kSeg);      // [kSeg]
-  __shared__ uint32_t used[kSeg / 32];
-  __shared__ int npos, nsingle;
+  __shared__ int npos_s, nsingle_s;
   const int bh = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s0 = blockIdx.x * kSeg, n = min(kSeg, nb - s0);
   const int32_t* S = sel + ((size_t)bh * nb + s0) * keep_k;
   int32_t* out = order + (size_t)bh * nb + s0;
   for (int e = threadIdx.x; e < kSeg * nwords; e += kThreads) bits[e] = 0u;
-  if (threadIdx.x < kSeg / 32) used[threadIdx.x] = 0u;
-  if (threadIdx.x == 0) { npos = 0; nsingle = 0; }
   __syncthreads();
-  for (int e = threadIdx.x; e < n * keep_k; e += kThreads) {
-    const int r = e / keep_k;
-    const int j = S[(size_t)r * keep_k + e % keep_k];
-    if (j >= 0 && j < nb) atomicOr(&bits[r * nwords + (j >> 5)], 1u << (j & 31));
+  // the segment's selections are n * keep_k consecutive entries; eight loads per thread are in
+  // flight before their atomics
+  const int total = n * keep_k;
+  for (int e0 = threadIdx.x; e0 < total; e0 += 8 * kThreads) {
+    int32_t jv[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) jv[x] = e0 + x * kThreads < total ? S[e0 + x * kThreads] : -1;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int j = jv[x];
+      if (j >= 0 && j < nb) atomicOr(&bits[(j >> 5) * kSeg + (e0 + x * kThreads) / keep_k], 1u << (j & 31));
+    }
   }
   __syncthreads();
+  // overlaps |S_x ∩ S_y| for x < y < n (the only entries the pass below reads)
   for (int e = threadIdx.x; e < kSeg * kSeg; e += kThreads) {
     const int x = e / kSeg, y = e % kSeg;
-    int cnt = 0;
     if (x < y && y < n) {
-      const uint32_t* bx = bits + x * nwords;
-      const uint32_t* by = bits + y * nwords;
-      for (int w = 0; w < nwords; ++w) cnt += __popc(bx[w] & by[w]);
+      int cnt = 0;
+      for (int w = 0; w < nwords; ++w) cnt += __popc(bits[w * kSeg + x] & bits[w * kSeg + y]);
+      ov[e] = (uint16_t)cnt;
     }
-    ov[e] = (uint16_t)cnt;
   }
   __syncthreads();
   if (warp == 0) {
+    // the set of paired blocks and the output counts stay in registers, identical in every lane
+    uint32_t u0 = 0u, u1 = 0u, u2 = 0u, u3 = 0u;
+    int npos = 0, nsingle = 0;
     for (int a = 0; a < n; ++a) {
-      if ((used[a >> 5] >> (a & 31)) & 1u) continue;
+      if (bit128(u0, u1, u2, u3, a)) continue;
       // best partner packed as ((overlap + 1) << 8) | (255 - distance): one warp max picks it (0 = none)
+      const uint16_t* row = ov + a * kSeg;
       uint32_t key = 0u;
-      for (int b = a + 1 + lane; b < n; b += 32) {
-        if (!((used[b >> 5] >> (b & 31)) & 1u))
-          key = max(key, ((uint32_t)(ov[a * kSeg + b] + 1) << 8) | (uint32_t)(255 - (b - a)));
+#pragma unroll
+      for (int x = 0; x < kSeg / 32; ++x) {
+        const int b = a + 1 + lane + 32 * x;
+        if (b < n && !bit128(u0, u1, u2, u3, b)) key = max(key, ((row[b] + 1u) << 8) | (uint32_t)(255 - (b - a)));
       }
       key = __reduce_max_sync(0xffffffffu, key);
-      if (lane == 0) {
-        used[a >> 5] |= 1u << (a & 31);
-        if (key) {
-          const int b = a + 255 - (int)(key & 255u);
-          used[b >> 5] |= 1u << (b & 31);
-          out[npos] = s0 + a;
-          out[npos + 1] = s0 + b;
-          npos += 2;
-        } else {
-          singles[nsingle++] = s0 + a;
-        }
+      const int pb = key ? a + 255 - (int)(key & 255u) : a;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int x = m ? pb : a;
+        const uint32_t bit = 1u << (x & 31);
+        const int w = x >> 5;
+        u0 |= w == 0 ? bit : 0u;
+        u1 |= w == 1 ? bit : 0u;
+        u2 |= w == 2 ? bit : 0u;
+        u3 |= w == 3 ? bit : 0u;
       }
-      __syncwarp();
+      if (key) {
+        if (lane == 0) {
+          out[npos] = s0 + a;
+          out[npos + 1] = s0 + pb;
+        }
+        npos += 2;
+      } else {
+        if (lane == 0) singles[nsingle] = s0 + a;
+        ++nsingle;
+      }
+    }
+    if (lane == 0) {
+      npos_s = npos;
+      nsingle_s = nsingle;
     }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < nsingle; e += kThreads) out[npos + e] = singles[e];
+  for (int e = threadIdx.x; e < nsingle_s; e += kThreads) out[npos_s + e] = singles[e];
 }
 
 __global__ void identity_order(int nb, int32_t* __restrict__ order) {
@@ -262,7 +314,7 @@ template <int D, int kRows>
 cudaError_t launch_route_kernel(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                                 float* scores, cudaStream_t stream) {
   const size_t smem = ((size_t)kRows * D + (size_t)tile_j<kRows>() * (D + 4) + (size_t)kRows * g.nb) * sizeof(float) +
-                      kWarps * 256 * sizeof(uint32_t) + kWarps * sizeof(float);
+                      kWarps * 256 * sizeof(uint32_t) + kWarps * sizeof(float) + (size_t)g.nb * sizeof(float);
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(route_kernel<D, kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
     return e;

@@ -234,33 +234,38 @@ __global__ void __launch_bounds__(kThreads) pair_kernel(const int32_t* __restric
   int32_t* out = order + (size_t)bh * nb + s0;
   for (int e = threadIdx.x; e < kSeg * nwords; e += kThreads) bits[e] = 0u;
   __syncthreads();
-  // the segment's selections are n * keep_k consecutive entries; eight loads per thread are in
+  // the segment's selections are n * keep_k consecutive entries; sixteen loads per thread are in
   // flight before their atomics
   const int total = n * keep_k;
-  for (int e0 = threadIdx.x; e0 < total; e0 += 8 * kThreads) {
-    int32_t jv[8];
+  for (int e0 = threadIdx.x; e0 < total; e0 += 16 * kThreads) {
+    int32_t jv[16];
 #pragma unroll
-    for (int x = 0; x < 8; ++x) jv[x] = e0 + x * kThreads < total ? S[e0 + x * kThreads] : -1;
+    for (int x = 0; x < 16; ++x) jv[x] = e0 + x * kThreads < total ? S[e0 + x * kThreads] : -1;
 #pragma unroll
-    for (int x = 0; x < 8; ++x) {
+    for (int x = 0; x < 16; ++x) {
       const int j = jv[x];
       if (j >= 0 && j < nb) atomicOr(&bits[(j >> 5) * kSeg + (e0 + x * kThreads) / keep_k], 1u << (j & 31));
     }
   }
   __syncthreads();
-  // overlaps |S_x ∩ S_y| for x < y < n (the only entries the pass below reads)
-  for (int e = threadIdx.x; e < kSeg * kSeg; e += kThreads) {
-    const int x = e / kSeg, y = e % kSeg;
-    if (x < y && y < n) {
+  // overlaps |S_x ∩ S_y| for x < y < n (the only entries the pass below reads): a warp per row x,
+  // its lanes over y
+  for (int x = warp; x < n; x += kWarps) {
+    for (int y = x + 1 + lane; y < n; y += 32) {
       int cnt = 0;
       for (int w = 0; w < nwords; ++w) cnt += __popc(bits[w * kSeg + x] & bits[w * kSeg + y]);
-      ov[e] = (uint16_t)cnt;
+      ov[x * kSeg + y] = (uint16_t)cnt;
     }
   }
   __syncthreads();
   if (warp == 0) {
-    // the set of paired blocks and the output counts stay in registers, identical in every lane
+    // The set of paired blocks and the output counts stay in registers: u0..u3 identical in every
+    // lane (for the test on a), and each lane's own view of its four blocks lane + 32 x (bit x of
+    // `avail` set while that block is unpaired), so a candidate test is one bit of one register.
     uint32_t u0 = 0u, u1 = 0u, u2 = 0u, u3 = 0u;
+    uint32_t avail = 0u;
+#pragma unroll
+    for (int x = 0; x < kSeg / 32; ++x) avail |= lane + 32 * x < n ? 1u << x : 0u;
     int npos = 0, nsingle = 0;
     for (int a = 0; a < n; ++a) {
       if (bit128(u0, u1, u2, u3, a)) continue;
@@ -269,11 +274,13 @@ __global__ void __launch_bounds__(kThreads) pair_kernel(const int32_t* __restric
       uint32_t key = 0u;
 #pragma unroll
       for (int x = 0; x < kSeg / 32; ++x) {
-        const int b = a + 1 + lane + 32 * x;
-        if (b < n && !bit128(u0, u1, u2, u3, b)) key = max(key, ((row[b] + 1u) << 8) | (uint32_t)(255 - (b - a)));
+        const int b = lane + 32 * x;
+        if (b > a && ((avail >> x) & 1u)) key = max(key, ((row[b] + 1u) << 8) | (uint32_t)(255 - (b - a)));
       }
       key = __reduce_max_sync(0xffffffffu, key);
       const int pb = key ? a + 255 - (int)(key & 255u) : a;
+      if (lane == (a & 31)) avail &= ~(1u << (a >> 5));
+      if (lane == (pb & 31)) avail &= ~(1u << (pb >> 5));
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const int x = m ? pb : a;

@@ -5,7 +5,6 @@ it can never complete.  The kernel must record PISA_DEVERR_WAIT_TIMEOUT in the w
 word within its (shortened) wait limit, drain its own work, free its tensor memory and return; the
 next call on the same context must then run normally and match the oracle.
 """
-import numpy as np
 import pytest
 import torch
 

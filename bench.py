@@ -315,6 +315,9 @@ def run_ours(args, rank, world, local_rank):
         "speedup_vs_dense_attention": round(dense_ms / attn_ms, 3),
         "exact_only_ms_per_attention_call": round(exact_only_ms, 4),
         "attention_overhead_vs_exact_only": round(attn_ms / exact_only_ms - 1.0, 4),
+        # the whole PISA step against the keep-or-drop attention call alone: an upper bound on the
+        # step overhead over an exact-only pipeline, whose own pre-compute and routing count as zero
+        "step_overhead_vs_exact_only_attention_alone": round((pre_ms + route_ms + attn_ms) / exact_only_ms - 1.0, 4),
         "effective_tflops_attention_only": round(exact_fl / (attn_ms * 1e-3) / 1e12, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": _profiled_traffic(w.name),

@@ -208,3 +208,21 @@ def test_reordering_entry_points_validate_without_launch():
     assert L.pisa_axis_permutation(2, 2, 3, 4, b"wth", out, 16) == C.PISA_OK
     got = list(out[:16])
     assert sorted(got) == list(range(16)) and got[12:] == [12, 13, 14, 15]
+
+
+def test_headers_are_plain_c_and_the_library_links_from_c(tmp_path):
+    """tests/c/abi_consumer.c: the public headers compile as strict C99 and a C program linked
+    against the library gets the same host-only answers as the binding (no GPU, no Python)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    libdir = os.path.dirname(C._LIB_PATH)
+    exe = str(tmp_path / "abi_consumer")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_consumer.c"), "-L", libdir, "-lpisa_b200",
+                    f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
+    res = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0, res.stderr
+    assert "c consumer ok: abi 5" in res.stdout

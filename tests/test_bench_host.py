@@ -20,3 +20,13 @@ def test_profiled_traffic_is_an_integer_or_none():
     t = bench._profiled_traffic("video-dit-large")
     assert t is None or (isinstance(t, int) and t > 0)
     assert bench._profiled_traffic("no-such-workload") is None
+
+
+def test_effective_flops_counts_selected_blocks_by_hand():
+    """4 d sum_i n_i sum_{j in S_i} cnt_j for the exact part, 4 d L (nb - keep_k) for the centroid
+    part, on a 150-token head with 64-token blocks (cnt = 64, 64, 22)."""
+    import torch
+    sel = torch.tensor([[[[0, 1], [1, 2], [0, 2]]]], dtype=torch.int32)
+    exact, centroid = bench.effective_flops(sel, 150, 64, 8, 3)
+    assert exact == 4 * 8 * (64 * (64 + 64) + 64 * (64 + 22) + 22 * (64 + 22))
+    assert centroid == 4 * 8 * 150 * (3 - 2)

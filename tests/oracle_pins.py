@@ -424,6 +424,45 @@ def pin_fp8_constant_key_blocks_are_dense():
     return worst < 1e-6, f"rel {worst:.2e}"
 
 
+def pin_fp8_correction_uses_unquantized_q():
+    """The e4m3 path quantizes only the logits: the first-order correction s (q_t Hbar) A_t / D_t
+    takes the unquantized q.  Two queries q1 and q1 + delta with the same e4m3 codes and row scales
+    (every row's largest entry, which sets its scale, is left alone; the others move by 1%, well
+    inside their rounding interval) give identical logits, so the outputs differ only through the
+    correction.  With keep_k = 0 and full blocks, A_t / D_t = sum_j alpha / sum_j cnt_j alpha =
+    1 / block for every row, so the difference is (s / block) delta Hbar exactly, with Hbar the
+    mean over blocks of cnt_j times the biased cross-covariance of the block's k and v (numpy.cov).
+    A correction built from the e4m3 copy of q would leave the two outputs equal."""
+    r = _rng(43)
+    L, d, block, scale = 64, 8, 16, 0.8
+    q1 = _representable(r, L, d, 0.003 * (1.0 + r.random(L)))
+    delta = 0.01 * q1
+    delta[:, 0] = 0.0                       # column 0 holds each row's largest |q| (the code 448)
+    k = r.standard_normal((L, d)) * 0.7
+    v = r.standard_normal((L, d))
+    hbar = np.zeros((d, d))
+    for s, e in O.block_bounds(L, block):
+        hbar += (e - s) * np.cov(k[s:e].T, v[s:e].T, bias=True)[:d, d:] / (L // block)
+    run = lambda qq: O.pisa_fp8(qq[None, None], k[None, None], v[None, None], block, 0, 0.5, scale)["o"][0, 0]
+    diff = run(q1 + delta) - run(q1)
+    want = (scale / block) * (delta @ hbar)
+    err = _rel(diff, want)
+    return bool(np.abs(want).max() > 0 and err < 1e-8), f"rel err {err:.3e}"
+
+
+def pin_dense_attention_is_sdpa():
+    """The oracle's textbook dense attention (used as the reference of the dense-attention checks)
+    equals torch SDPA in float64, with d != dv, a scale, and logits large enough that an unshifted
+    exponential would overflow."""
+    worst = 0.0
+    for seed, (L, Lk, d, dv), scale, spread in ((50, (37, 53, 6, 4), 0.7, 1.0), (51, (64, 64, 16, 16), 1.0, 9.0)):
+        q, k, _ = _qkv(seed, L, d, spread=spread)
+        k = _rng(seed + 100).standard_normal((Lk, d)) * spread
+        v = _rng(seed + 200).standard_normal((Lk, dv))
+        worst = max(worst, _rel(O.dense_attention(q, k, v, scale), _sdpa(q, k, v, scale)))
+    return worst < 1e-12, f"max rel err {worst:.3e}"
+
+
 ALL_PINS = [
     pin_all_selected_is_dense, pin_block_one_is_dense, pin_constant_key_blocks_are_dense,
     pin_exact_only_is_masked_sdpa, pin_brute_force_matches, pin_value_shift_equivariance,
@@ -434,5 +473,5 @@ ALL_PINS = [
     pin_axis_permutation_by_hand, pin_axis_permutation_coordinates,
     pin_permute_rows_inverse_and_dense_equivariance, pin_reordered_pisa_all_selected_is_dense,
     pin_e4m3_by_hand, pin_quantize_groups_bounds, pin_fp8_exact_on_representable_inputs,
-    pin_fp8_constant_key_blocks_are_dense,
+    pin_fp8_constant_key_blocks_are_dense, pin_fp8_correction_uses_unquantized_q, pin_dense_attention_is_sdpa,
 ]

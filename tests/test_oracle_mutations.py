@@ -99,6 +99,23 @@ _ORIG["fp8_logit_inputs"] = O.fp8_logit_inputs
 _ORIG["e4m3"] = O.e4m3
 
 
+
+def _corr_from_logit_q(*args, q_corr=None, **kw):
+    # the e4m3 path's correction built from the quantized q that the logits use
+    return _ORIG["attention_head"](*args, **kw)
+
+
+def _dense_wrong_axis(q, k, v, scale=1.0):
+    s = scale * (np.asarray(q, np.float64) @ np.asarray(k, np.float64).T)
+    p = np.exp(s - s.max(axis=0, keepdims=True))
+    return (p / p.sum(axis=0, keepdims=True)) @ np.asarray(v, np.float64)
+
+
+MUTATIONS["e4m3 correction uses the quantized q"] = ("attention_head", _corr_from_logit_q)
+MUTATIONS["dense attention normalised over queries"] = ("dense_attention", _dense_wrong_axis)
+_ORIG["attention_head"] = O.attention_head
+_ORIG["dense_attention"] = O.dense_attention
+
 def _caught():
     failed = []
     for pin in P.ALL_PINS:

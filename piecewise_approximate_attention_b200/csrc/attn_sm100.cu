@@ -244,7 +244,8 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
-      if (p.fault != 1) {      // fault 1 (tests only): never load Q, so the MMA warp's wait runs out
+      const bool issued_q = p.fault != 1;   // fault 1 (tests only): never load Q, so the MMA warp's wait runs out
+      if (issued_q) {
         if (kF8) {             // e4m3 Q: one 128-byte row per token, 16 KB
           mbar_expect_tx(&sm.bar_q, kHalf);
           tma_load_3d(sm.q, &maps.q8, &sm.bar_q, 0, qa * p.block, bh);
@@ -344,15 +345,12 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
       }
       {
         // drain: every copy issued must land before this CTA's shared memory is released (in a
-        // normal run the MMA warp has waited for all of them, so these waits return at once)
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
-        if (issued_q16)
-          while (!mbar_try_wait(&sm.bar_q16, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
-        for (int i = max(0, issued_k - kKS); i < issued_k; ++i)
-          while (!mbar_try_wait(&sm.bar_kfull[i % kKS], (i / kKS) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
-        for (int i = max(0, issued_v - kVS); i < issued_v; ++i)
-          while (!mbar_try_wait(&sm.bar_vfull[i % kVS], (i / kVS) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+        // normal run the MMA warp has waited for all of them, so these waits return at once).
+        // Each wait has its own deadline, so one that gives up cannot cut the others short.
+        if (issued_q) mbar_drain(&sm.bar_q, 0, p.wait_ns);
+        if (issued_q16) mbar_drain(&sm.bar_q16, 0, p.wait_ns);
+        for (int i = max(0, issued_k - kKS); i < issued_k; ++i) mbar_drain(&sm.bar_kfull[i % kKS], (i / kKS) & 1, p.wait_ns);
+        for (int i = max(0, issued_v - kVS); i < issued_v; ++i) mbar_drain(&sm.bar_vfull[i % kVS], (i / kVS) & 1, p.wait_ns);
       }
     }
   } else if (warp == 5) {

@@ -225,12 +225,10 @@ perblock_sm100(const __grid_constant__ AttnMaps maps, const __grid_constant__ CU
       {
         // every copy issued must land before this CTA's shared memory is released (normally the
         // MMA warp has already waited for all of them)
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&sm.bar_q, 0) && globaltimer_ns() - t0 < p.wait_ns) {}
-        if (issued_k > 0)
-          while (!mbar_try_wait(&sm.bar_kfull, (issued_k - 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
-        for (int i = max(0, issued_h - kR); i < issued_h; ++i)
-          while (!mbar_try_wait(&sm.bar_full[i % kR], (i / kR) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+        // (each wait with its own deadline)
+        mbar_drain(&sm.bar_q, 0, p.wait_ns);
+        if (issued_k > 0) mbar_drain(&sm.bar_kfull, (issued_k - 1) & 1, p.wait_ns);
+        for (int i = max(0, issued_h - kR); i < issued_h; ++i) mbar_drain(&sm.bar_full[i % kR], (i / kR) & 1, p.wait_ns);
       }
     }
   } else if (warp == 5) {

@@ -76,6 +76,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Waits, for at most `limit_ns` of its own, for the phase with the given parity to complete (a
+// drain before shared memory or tensor memory is released: no abort flag, nothing recorded).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < limit_ns) {}
+}
+
 // ---------------------------------------------------------------------------------------------
 // TMA (tiled, no multicast)
 // ---------------------------------------------------------------------------------------------

@@ -1,12 +1,15 @@
 """Benchmark of the PISA hot path (pre-compute -> route -> attention) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+    python bench.py --profile-case [--workload NAME] [--heads H] [--iters I] [--mode pisa|per_block]
+                    [--dtype bf16|bf16_fp8qk] [--reorder AXES]
 
 One step = one pass of the three calls over one batch of synthetic, device-resident input.  The
 metric is effective TFLOP/s (FLOPs of the exactly-attended, selected blocks only) per step, summed
 over ranks; each rank runs its own batch element (weak scaling, no data-path collective).  Rank 0
 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample
-of the same workload, on the host cores.
+of the same workload, on the host cores.  ``--profile-case`` only runs the hot path a few times on
+a slice of a workload (no timing, no JSON), for a profiler such as ncu to capture.
 """
 from __future__ import annotations
 
@@ -110,6 +113,90 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+class NvmlClock:
+    """SM clock of one GPU sampled every 2 ms by NVML in a background thread, so that each timed
+    call can be given the median clock seen while it ran (host time window around the call)."""
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.stop_flag = False
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+        except Exception:
+            self.nvml = None
+
+    def __enter__(self):
+        import threading
+        if self.nvml is not None:
+            def poll():
+                while not self.stop_flag:
+                    self.samples.append((time.perf_counter(),
+                                         self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)))
+                    time.sleep(0.002)
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self.stop_flag = True
+        if self.thread is not None:
+            self.thread.join(timeout=1)
+
+    def window(self, t0: float, t1: float):
+        v = [c for (t, c) in self.samples if t0 <= t <= t1]
+        return float(statistics.median(v)) if v else None
+
+
+def time_arms(arms, reps: int, stream, clock=None, every=None, warmup: int = 2):
+    """Interleaved timing: rep r runs every arm once, in order (A B C A B C ...), each call bracketed
+    by CUDA events on `stream` and a synchronize, so that the arms share the GPU's clock and thermal
+    state.  ``every[name] = n`` runs that arm only on every n-th rep.  Returns {name: [(ms, MHz)]}."""
+    import torch
+    every = every or {}
+    for fn in arms.values():
+        for _ in range(warmup):
+            fn()
+    torch.cuda.synchronize()
+    out = {name: [] for name in arms}
+    for r in range(reps):
+        for name, fn in arms.items():
+            if r % every.get(name, 1):
+                continue
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            t0 = time.perf_counter()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            t1 = time.perf_counter()
+            out[name].append((e0.elapsed_time(e1), clock.window(t0, t1) if clock is not None else None))
+    return out
+
+
+def _pct(xs, q):
+    import numpy as np
+    return float(np.percentile(np.asarray(xs, dtype=np.float64), q))
+
+
+def summarize(samples):
+    """Median, 10th and 90th percentile of the times (ms), median SM clock and sample count."""
+    ms = [m for m, _ in samples]
+    mhz = [c for _, c in samples if c is not None]
+    return {"median_ms": round(_pct(ms, 50), 4), "p10_ms": round(_pct(ms, 10), 4), "p90_ms": round(_pct(ms, 90), 4),
+            "sm_mhz": round(statistics.median(mhz), 1) if mhz else None, "n": len(ms)}
+
+
+def ratio_summary(num, den):
+    """Per-rep ratio num_r / den_r - 1 of two interleaved arms: median, p10, p90."""
+    rs = [a[0] / b[0] - 1.0 for a, b in zip(num, den)]
+    return {"median": round(_pct(rs, 50), 4), "p10": round(_pct(rs, 10), 4), "p90": round(_pct(rs, 90), 4), "n": len(rs)}
+
+
 def effective_flops(sel, order_blocks_L: int, block: int, d: int, nb: int):
     """(exact FLOPs of selected blocks, centroid FLOPs of unselected blocks) for sel [B,H,nqb,k]."""
     import torch
@@ -211,10 +298,46 @@ def run_ours(args, rank, world, local_rank):
     ms_step = total_ms / args.steps
     (ms_step, attn_ms_max), (exact_all,) = aggregate([ms_step, attn_ms], [exact_fl], dev, world)
 
-    # library's own dense path (keep_k = nb) and exact-only mode, same GPU, outside the timed region
+    # Outside the timed region, interleaved on the same GPU (A B C D ... per rep): PISA against the
+    # exact-only (keep-or-drop) pipeline, whose pre-computation writes the zeroth-order statistics
+    # only and whose routing drops the covariance term (lambda = 0), and against the library's
+    # dense path (keep_k = nb).
     dense = Pisa(B, H, L, d, w.block, p.nb, w.lam, w.dtype, 1.0, dev, pair=False)
     dense.precompute(qd, kd, vd, stream)
     dense.route(stream=stream)
+    x = Pisa(B, H, L, d, w.block, w.keep_k, 0.0, w.dtype, 1.0, dev, C.PISA_MODE_EXACT_ONLY, first_order=False)
+    o2 = torch.empty_like(o)
+    arms = {
+        "pisa_step": lambda: (p.precompute(qd, kd, vd, stream), p.route(stream=stream),
+                              p.attention(qd, kd, vd, o2, stream=stream)),
+        "exact_only_step": lambda: (x.precompute(qd, kd, vd, stream), x.route(stream=stream),
+                                    x.attention(qd, kd, vd, o2, stream=stream)),
+        "pisa_attention": lambda: p.attention(qd, kd, vd, o2, stream=stream),
+        "exact_only_attention_same_selection": lambda: p.attention(qd, kd, vd, o2, mode=C.PISA_MODE_EXACT_ONLY,
+                                                                   stream=stream),
+        "pisa_precompute": lambda: p.precompute(qd, kd, vd, stream),
+        "zeroth_order_precompute": lambda: x.precompute(qd, kd, vd, stream),
+        "pisa_route": lambda: p.route(stream=stream),
+        "lambda0_route": lambda: x.route(stream=stream),
+        "dense_attention": lambda: dense.attention(qd, kd, vd, o2, stream=stream),
+    }
+    with NvmlClock(local_rank) as nclk:
+        raw = time_arms(arms, args.arm_reps, stream, nclk, every={"dense_attention": 4})
+    torch.cuda.synchronize()
+    st_x, code_x = x.device_error(stream)
+    if st_x != C.PISA_OK:
+        raise RuntimeError(f"device status {st_x} code {code_x} in the exact-only pipeline")
+    arm_stats = {name: summarize(v) for name, v in raw.items()}
+    dense_ms = arm_stats["dense_attention"]["median_ms"]
+    exact_only_ms = arm_stats["exact_only_attention_same_selection"]["median_ms"]
+    overhead = {
+        "definition": "(T_pre + T_route + T_attn, PISA) / (T_pre, zeroth order + T_route, lambda 0 + T_attn, "
+                      "keep-or-drop) - 1, each rep's two steps timed back to back",
+        "pipeline": ratio_summary(raw["pisa_step"], raw["exact_only_step"]),
+        "attention_same_selection": ratio_summary(raw["pisa_attention"], raw["exact_only_attention_same_selection"]),
+        "target": 0.15,
+    }
+    del x
 
     def time_calls(fn, n=3):
         fn()
@@ -227,10 +350,9 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / n
 
-    o2 = torch.empty_like(o)
-    dense_ms = time_calls(lambda: dense.attention(qd, kd, vd, o2, stream=stream))
+    dense.attention(qd, kd, vd, o2, stream=stream)
     o_dense = o2.clone()
-    exact_only_ms = time_calls(lambda: p.attention(qd, kd, vd, o2, mode=C.PISA_MODE_EXACT_ONLY, stream=stream))
+    p.attention(qd, kd, vd, o2, mode=C.PISA_MODE_EXACT_ONLY, stream=stream)
     rel_keep_or_drop = rel_l2(o2, o_dense)
     dense_fl = 4.0 * L * L * d * B * H
     del dense
@@ -239,6 +361,7 @@ def run_ours(args, rank, world, local_rank):
     reordering = token_reordering(p, w, (qd, kd, vd), o_dense, stream, time_calls) if not args.no_extras else None
     del o_dense
     short = short_sequences(dev) if not args.no_extras else None
+    sweep_result = sweep(dev, args.sweep_reps) if not args.no_extras and args.sweep_reps > 0 else None
 
     # end to end through the public API with host buffers: H2D of q, k, v and D2H of o every step
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
@@ -312,12 +435,10 @@ def run_ours(args, rank, world, local_rank):
         "ms_route": round(route_ms, 4),
         "dense_ms_per_attention_call": round(dense_ms, 4),
         "dense_tflops": round(dense_fl / (dense_ms * 1e-3) / 1e12, 3),
-        "speedup_vs_dense_attention": round(dense_ms / attn_ms, 3),
+        "speedup_vs_dense_attention": round(dense_ms / arm_stats["pisa_attention"]["median_ms"], 3),
         "exact_only_ms_per_attention_call": round(exact_only_ms, 4),
-        "attention_overhead_vs_exact_only": round(attn_ms / exact_only_ms - 1.0, 4),
-        # the whole PISA step against the keep-or-drop attention call alone: an upper bound on the
-        # step overhead over an exact-only pipeline, whose own pre-compute and routing count as zero
-        "step_overhead_vs_exact_only_attention_alone": round((pre_ms + route_ms + attn_ms) / exact_only_ms - 1.0, 4),
+        "overhead_vs_exact_only_pipeline": overhead,
+        "arms": arm_stats,
         "effective_tflops_attention_only": round(exact_fl / (attn_ms * 1e-3) / 1e12, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": _profiled_traffic(w.name),
@@ -336,6 +457,7 @@ def run_ours(args, rank, world, local_rank):
         "per_block_first_order": per_block,
         "short_sequences": short,
         "token_reordering": reordering,
+        "sweep": sweep_result,
     }
     if rank == 0:
         result["cpu_baseline"] = cpu_baseline(w)
@@ -449,50 +571,105 @@ def run_step_reordered(p, qkv, buf, o_r, o, perm, stream):
 SHORT_WORKLOADS = ("image-dit", "sweep-L8192-s0.875")
 
 
-def short_sequences(dev, steps: int = 20):
+def short_sequences(dev, reps: int = 30):
     """Short sequences, where per-launch overhead and the pre-computation weigh most: the full
     step (pre-compute + route + attention) launched call by call and replayed as one CUDA graph,
-    its parts, and the library's dense attention on the same inputs.  Outside the timed region."""
+    its parts, and the library's dense attention on the same inputs, timed interleaved (medians).
+    Outside the timed region."""
     import torch
     from piecewise_approximate_attention_b200.runtime import Pisa
     from piecewise_approximate_attention_b200.workloads import WORKLOADS, make_qkv
     out = {}
+    stream = torch.cuda.current_stream(dev)
     for name in SHORT_WORKLOADS:
         w = WORKLOADS[name]
         q, k, v = (x.to(dev) for x in make_qkv(w))
         B, H, L, d = q.shape
         p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, dev)
         o = torch.empty_like(q)
-        ev = lambda: torch.cuda.Event(enable_timing=True)
-
-        def timed(fn):
-            for _ in range(3):
-                fn()
-            a, b = ev(), ev()
-            torch.cuda.synchronize()
-            a.record()
-            for _ in range(steps):
-                fn()
-            b.record()
-            torch.cuda.synchronize()
-            return a.elapsed_time(b) / steps
-
-        direct = timed(lambda: p(q, k, v, o))
-        pre = timed(lambda: p.precompute(q, k, v))
-        route = timed(lambda: p.route())
-        attn = timed(lambda: p.attention(q, k, v, o))
         graph = p.capture(q, k, v, o)
-        replay = timed(graph.replay)
         dense = Pisa(B, H, L, d, w.block, p.nb, w.lam, w.dtype, 1.0, dev, pair=False)
         dense.precompute(q, k, v)
         dense.route()
-        dense_ms = timed(lambda: dense.attention(q, k, v, o))
+        arms = {"step_launches": lambda: p(q, k, v, o), "step_graph": graph.replay,
+                "precompute": lambda: p.precompute(q, k, v), "route": lambda: p.route(),
+                "attention": lambda: p.attention(q, k, v, o), "dense_attention": lambda: dense.attention(q, k, v, o)}
+        with NvmlClock(dev.index or 0) as nclk:
+            raw = time_arms(arms, reps, stream, nclk)
+        st = {a: summarize(v) for a, v in raw.items()}
         out[name] = {"seq_len": L, "heads": H, "keep_k": w.keep_k, "num_blocks": p.nb,
-                     "ms_step_launches": round(direct, 4), "ms_step_graph": round(replay, 4),
-                     "ms_precompute": round(pre, 4), "ms_route": round(route, 4), "ms_attention": round(attn, 4),
-                     "ms_dense_attention": round(dense_ms, 4),
-                     "speedup_step_vs_dense": round(dense_ms / replay, 3)}
+                     **{f"ms_{a}": st[a]["median_ms"] for a in arms},
+                     "p10_p90_ms_step_graph": [st["step_graph"]["p10_ms"], st["step_graph"]["p90_ms"]],
+                     "sm_mhz": st["step_graph"]["sm_mhz"],
+                     "speedup_step_vs_dense": round(st["dense_attention"]["median_ms"] / st["step_graph"]["median_ms"], 3)}
         del graph, p, dense
+    return out
+
+
+SWEEP_GRIDS = ((8, 32, 32), (32, 32, 32), (32, 64, 64))
+SWEEP_KEEP = (0.5, 0.25, 0.125, 0.0625)
+
+
+def sweep(dev, reps: int = 5, seeds=(0, 1, 2)):
+    """Sequence length x density sweep (16 heads, head_dim 128, bf16, block 64; L 8192, 32768 and
+    131072 on 8x32x32, 32x32x32 and 32x64x64 grids; keep 1/2, 1/4, 1/8 and 1/16 of the key blocks
+    per query block, and all of them), seeds 0-2.  Per point, over seeds and reps (interleaved with
+    the dense call): the whole step (pre-compute + route + attention), the attention call, the
+    library's dense attention (keep_k = nb) and the speedups, as median [p10, p90].  Outside the
+    timed region."""
+    import math
+
+    import torch
+    from piecewise_approximate_attention_b200.runtime import Pisa
+    from piecewise_approximate_attention_b200.workloads import Workload, make_qkv
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for grid in SWEEP_GRIDS:
+        L = grid[0] * grid[1] * grid[2]
+        acc = {}
+        for seed in seeds:
+            w = Workload(f"sweep-L{L}", 1, 16, grid, 0, 128, 64, 0.0, 0.5, "bf16", seed=seed)
+            q, k, v = (x.to(dev) for x in make_qkv(w))
+            nb = w.num_blocks
+            o = torch.empty_like(q)
+            dense = Pisa(1, 16, L, 128, 64, nb, 0.5, "bf16", 1.0, dev, pair=False)
+            dense.precompute(q, k, v)
+            dense.route()
+            pis = {}
+            arms = {"dense_attention": lambda: dense.attention(q, k, v, o),
+                    "dense_step": lambda: dense(q, k, v, o)}
+            for frac in SWEEP_KEEP:
+                keep = int(math.ceil(frac * nb - 1e-9))
+                pis[frac] = Pisa(1, 16, L, 128, 64, keep, 0.5, "bf16", 1.0, dev)
+                pis[frac].precompute(q, k, v)
+                pis[frac].route()
+                arms[f"step_{frac:g}"] = (lambda pp: lambda: pp(q, k, v, o))(pis[frac])
+                arms[f"attention_{frac:g}"] = (lambda pp: lambda: pp.attention(q, k, v, o))(pis[frac])
+            raw = time_arms(arms, reps, stream, warmup=1)
+            for a, vals in raw.items():
+                acc.setdefault(a, []).extend(vals)
+            for pp in pis.values():
+                if pp.device_error() != (0, 0):
+                    raise RuntimeError("device status set in the sweep")
+            del pis, dense, q, k, v, o
+            torch.cuda.empty_cache()
+
+        def med(a):
+            return [round(_pct([m for m, _ in acc[a]], x), 4) for x in (50, 10, 90)]
+
+        dn = statistics.median(m for m, _ in acc["dense_attention"])
+        row = {"num_blocks": -(-L // 64), "dense": {"keep_k": -(-L // 64), "step_ms": med("dense_step"),
+                                                    "attention_ms": med("dense_attention")}}
+        for frac in SWEEP_KEEP:
+            st = statistics.median(m for m, _ in acc[f"step_{frac:g}"])
+            at = statistics.median(m for m, _ in acc[f"attention_{frac:g}"])
+            row[f"keep_{frac:g}"] = {"keep_k": int(math.ceil(frac * (-(-L // 64)) - 1e-9)),
+                                     "step_ms": med(f"step_{frac:g}"), "attention_ms": med(f"attention_{frac:g}"),
+                                     "speedup_attention_vs_dense": round(dn / at, 3),
+                                     "speedup_step_vs_dense": round(dn / st, 3)}
+        out[f"L{L}"] = row
+    out["note"] = ("step = pre-compute + route + attention launched call by call; times are medians "
+                   "[p10, p90] over seeds 0-2 x reps, interleaved with the dense call; dense = keep_k = nb")
     return out
 
 
@@ -549,6 +726,40 @@ def run_reference(args, rank, world):
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def profile_case(a):
+    """Runs the hot path a few times on a slice of a workload and nothing else: the command that
+    the ncu captures summarised under profiles/ run (no timing, no JSON line)."""
+    import torch
+    from piecewise_approximate_attention_b200 import _lib as C
+    from piecewise_approximate_attention_b200.runtime import Pisa, reorder_tokens, restore_tokens
+    from piecewise_approximate_attention_b200.workloads import WORKLOADS, make_qkv
+    mode = C.PISA_MODE_PER_BLOCK if a.mode == "per_block" else C.PISA_MODE_PISA
+    w = WORKLOADS[a.workload].with_(heads=a.heads)
+    q, k, v = (x.cuda() for x in make_qkv(w))
+    B, H, L, d = q.shape
+    p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, a.dtype, 1.0, "cuda", mode)
+    o = torch.empty_like(q)
+    perm = None
+    if a.reorder:
+        perm = torch.from_numpy(C.pisa_axis_permutation(w.grid, a.reorder, w.text_tokens)).cuda()
+        bufs = [torch.empty_like(q) for _ in range(3)]
+        o_r = torch.empty_like(q)
+    for _ in range(a.iters):
+        if perm is None:
+            p(q, k, v, o)
+        else:
+            for x, b in zip((q, k, v), bufs):
+                reorder_tokens(x, perm, out=b)
+            p(*bufs, o_r)
+            restore_tokens(o_r, perm, out=o)
+    torch.cuda.synchronize()
+    st = p.device_error()
+    print(f"{w.name} heads={H} L={L} block={w.block} keep_k={w.keep_k} mode={a.mode} dtype={a.dtype} "
+          f"reorder={a.reorder} iters={a.iters} status={st}")
+    if st[0] != 0:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -556,10 +767,23 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--no-extras", action="store_true", help="skip the short-sequence measurements")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the token-reordering, short-sequence and sweep measurements")
+    ap.add_argument("--arm-reps", type=int, default=20, help="interleaved reps of each comparison arm")
+    ap.add_argument("--sweep-reps", type=int, default=4, help="reps per seed of the length x density sweep")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="only run the hot path --iters times on --heads heads of --workload (for ncu)")
+    ap.add_argument("--heads", type=int, default=8)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--mode", choices=("pisa", "per_block"), default="pisa")
+    ap.add_argument("--dtype", choices=("bf16", "bf16_fp8qk"), default="bf16")
+    ap.add_argument("--reorder", default=None, help="axis order of the frames x height x width grid, e.g. hwt")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    if args.profile_case:
+        profile_case(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

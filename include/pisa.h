@@ -148,16 +148,32 @@ PISA_API size_t pisa_perblock_workspace_bytes(const pisa_shape* shape);
 PISA_API pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
                             const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream);
 
+/* Zeroth-order pre-computation: the part of pisa_precompute that the zeroth-order Taylor term and
+ * routing without the covariance term need (§2 핵심 알고리즘, zeroth-order bullet: block centroids
+ * and value sums; the pooled queries of 공분산 인식 라우팅).  Writes qbar, kbar and vsum and, for
+ * bf16 inputs, kbar_op, vsum_op, v_op and vscale (and the e4m3 copies for PISA_BF16_FP8QK); leaves
+ * hbar, M, hbar_op, H and hdiff_op unwritten.  The statistics it writes equal pisa_precompute's bit
+ * for bit.  What they serve: pisa_route with lambda == 0 (which does not read M) and pisa_attention
+ * in PISA_MODE_EXACT_ONLY, i.e. a keep-or-drop pipeline, the baseline the method is measured
+ * against (§1 문제 정의); PISA_MODE_PISA and PISA_MODE_PER_BLOCK need the full pisa_precompute.
+ * It reads q, k and v once (no second pass over k and v, no first-order contractions).  Arguments,
+ * ws and errors as for pisa_precompute. */
+PISA_API pisa_status pisa_precompute_zeroth_order(const pisa_shape* shape, const void* q, const void* k,
+                                                  const void* v, const pisa_stats* stats, void* ws,
+                                                  size_t ws_bytes, pisa_stream_t stream);
+
 /* pisa_precompute without a caller workspace, for callers that cannot allocate device memory (a
  * plugin whose host framework owns every device allocation, or a path that must not call cudaMalloc
  * because it may synchronise the device).  The method's description has no counterpart to this call;
  * it exists for such callers.  It runs the same kernels as pisa_precompute, with the scratch taken
  * from a fixed 16 MiB array in the library's device memory, which every device that loads the
  * library holds until the process exits.  It allocates nothing and frees nothing.
- *   - Shapes whose pisa_workspace_bytes exceeds 16 MiB return PISA_ERR_UNSUPPORTED and enqueue
- *     nothing; other invalid arguments are rejected exactly as by pisa_precompute.
- *   - The first call on a device looks up the array's device address on that device (a host-side
- *     CUDA runtime query); make that first call before any stream capture.
+ *   - Arguments are checked first, exactly as by pisa_precompute (it takes no workspace, so there
+ *     is no workspace check); then shapes whose pisa_workspace_bytes exceeds 16 MiB return
+ *     PISA_ERR_UNSUPPORTED.  A rejected call enqueues nothing and does not touch the array.
+ *   - The first call in a device's CUDA context looks up the array's device address there (a
+ *     host-side CUDA runtime query); make that first call before any stream capture.  If the
+ *     context is replaced (cudaDeviceReset), the next call looks the address up again.
  *   - Every call, on any stream, shares the one array: calls that overlap on the GPU race.  Each
  *     call clears the status word it uses before its kernels start; device-side wait timeouts of
  *     this call are not reported to the caller.
@@ -174,7 +190,8 @@ PISA_API pisa_status pisa_precompute_noalloc(const pisa_shape* shape, const void
  *        with similar selections next to each other (pisa_attention runs consecutive pairs of it as
  *        one 128-row tile when block == 64; it changes no result).
  * scores nullable [B,H,nb,nb] fp32: r_ij.
- * Requires 0 <= keep_k <= nb, lambda finite and >= 0, nb <= 4096. */
+ * Requires 0 <= keep_k <= nb, lambda finite and >= 0, nb <= 4096.  With lambda == 0 the M term is
+ * dropped and stats->M is not read (it may be unwritten, as after pisa_precompute_zeroth_order). */
 PISA_API pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,
                        int32_t* sel, int32_t* order, float* scores, pisa_stream_t stream);
 

@@ -21,7 +21,7 @@ PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
            "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string",
            "pisa_precompute_noalloc", "pisa_testing_set_attention_fault", "pisa_perblock_workspace_bytes",
-           "pisa_permute_rows", "pisa_axis_permutation")
+           "pisa_permute_rows", "pisa_axis_permutation", "pisa_precompute_zeroth_order")
 
 
 class PisaShape(ctypes.Structure):
@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
             "pisa_workspace_bytes": (sz, [P(PisaShape)]),
             "pisa_perblock_workspace_bytes": (sz, [P(PisaShape)]),
             "pisa_precompute": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, sz, vp]),
+            "pisa_precompute_zeroth_order": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, sz, vp]),
             "pisa_route": (i32, [P(PisaShape), P(PisaStats), i32, f32, vp, vp, vp, vp]),
             "pisa_attention": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, vp, i32, i32, vp, vp, sz, vp]),
             "pisa_read_device_error": (i32, [vp, P(i32), vp]),
@@ -201,6 +202,12 @@ def alloc_workspace(shape: PisaShape, device, per_block: bool = False):
 def pisa_precompute(shape: PisaShape, q, k, v, stats: Stats, ws, stream=None):
     _check(lib().pisa_precompute(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(stats.c), _ptr(ws),
                                  ws.numel(), _stream(stream)), "pisa_precompute")
+
+
+def pisa_precompute_zeroth_order(shape: PisaShape, q, k, v, stats: Stats, ws, stream=None):
+    """Zeroth-order statistics only (what lambda = 0 routing and the keep-or-drop mode read)."""
+    _check(lib().pisa_precompute_zeroth_order(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(stats.c),
+                                              _ptr(ws), ws.numel(), _stream(stream)), "pisa_precompute_zeroth_order")
 
 
 def pisa_precompute_noalloc(shape: PisaShape, q, k, v, stats: Stats, stream=None):

@@ -92,13 +92,22 @@ void stats_sizes(const Dims& g, int with_H, size_t out[kStatsArrays]) {
 }
 
 }  // namespace
+
+pisa_status validate_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                                const pisa_stats* stats, Dims* g) {
+  pisa_status s = check_shape(shape, g);
+  if (s != PISA_OK) return s;
+  if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return PISA_ERR_INVALID_ARG;
+  return check_stats(*g, stats, true);
+}
+
 }  // namespace pisa
 
 using namespace pisa;
 
 extern "C" {
 
-int32_t pisa_abi_version(void) { return 5; }
+int32_t pisa_abi_version(void) { return 6; }
 
 int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
   if (seq_len < 1 || block < 1) return -1;
@@ -168,22 +177,31 @@ size_t pisa_perblock_workspace_bytes(const pisa_shape* shape) {
   return pb > base ? pb : base;
 }
 
-pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
-                            const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+namespace {
+pisa_status precompute(const pisa_shape* shape, const void* q, const void* k, const void* v, const pisa_stats* stats,
+                       void* ws, size_t ws_bytes, bool first_order, pisa_stream_t stream) {
   Dims g;
-  pisa_status s = check_shape(shape, &g);
+  pisa_status s = validate_precompute(shape, q, k, v, stats, &g);
   if (s != PISA_OK) return s;
-  if (!q || !k || !v || !ws || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(ws))
-    return PISA_ERR_INVALID_ARG;
-  if ((s = check_stats(g, stats, true)) != PISA_OK) return s;
-  if (ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (bf16_inputs(g.dtype)) {
-    cudaError_t e = launch_precompute_sm100(g, q, k, v, *stats, ws, cs);
+    cudaError_t e = launch_precompute_sm100(g, q, k, v, *stats, ws, first_order, cs);
     if (e == cudaSuccess && g.dtype == PISA_BF16_FP8QK) e = launch_quantize_fp8(g, q, k, *stats, cs);
     return cuda_status(e);
   }
-  return cuda_status(launch_precompute_simt(g, q, k, v, *stats, ws, cs));
+  return cuda_status(launch_precompute_simt(g, q, k, v, *stats, ws, first_order, cs));
+}
+}  // namespace
+
+pisa_status pisa_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                            const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+  return precompute(shape, q, k, v, stats, ws, ws_bytes, true, stream);
+}
+
+pisa_status pisa_precompute_zeroth_order(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                                         const pisa_stats* stats, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+  return precompute(shape, q, k, v, stats, ws, ws_bytes, false, stream);
 }
 
 pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,

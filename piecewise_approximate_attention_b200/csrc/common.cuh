@@ -84,11 +84,17 @@ bool encode_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t r
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits: 2 s
 
+// Argument checks of pisa_precompute other than its workspace (shape, q, k, v, stats); fills *g.
+// Enqueues nothing.  Shared by the entry points that run the pre-computation.
+pisa_status validate_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                                const pisa_stats* stats, Dims* g);
+
 // ---- launchers (defined in the kernel translation units) ----
+// first_order = false: the zeroth-order statistics only (pisa_precompute_zeroth_order).
 cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,
-                                   const pisa_stats& st, void* ws, cudaStream_t stream);
+                                   const pisa_stats& st, void* ws, bool first_order, cudaStream_t stream);
 cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v,
-                                    const pisa_stats& st, void* ws, cudaStream_t stream);
+                                    const pisa_stats& st, void* ws, bool first_order, cudaStream_t stream);
 cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const float* vmax,
                                const pisa_stats& st, cudaStream_t stream);
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,

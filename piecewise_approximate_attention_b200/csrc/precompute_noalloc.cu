@@ -8,8 +8,11 @@
 //
 // The array is a file-scope __device__ variable of kNoAllocScratchBytes.  Every device on which the
 // library's module is loaded holds it until the process exits.  In host code its name is only a
-// host-side stand-in, so the device address is looked up with cudaGetSymbolAddress, once per device,
-// with that device current, on the first call made on that device.
+// host-side stand-in, so its device address is looked up with cudaGetSymbolAddress, with the device
+// current, the first time a call runs in a device's CUDA context (and again if that context has been
+// replaced, e.g. after cudaDeviceReset, since the module is then loaded afresh).
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -23,22 +26,55 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+struct ScratchEntry {
+  unsigned long long ctx_id = 0;   // CUDA context the address belongs to (0 = not looked up yet)
+  void* addr = nullptr;
+};
+ScratchEntry g_scratch[kMaxDevices];
 
-// Device address of g_noalloc_scratch on the current device (looked up once per device).
+// Unique id of the calling thread's current CUDA context (0 if none is current or the driver
+// cannot say).  Driver entry points through the runtime: no link-time dependency on libcuda.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch in the current device's context.  Looked up once per
+// context; a host-side query that allocates nothing.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  ScratchEntry& ent = g_scratch[dev];
+  const unsigned long long id = current_context_id();
+  if (!ent.addr || id == 0 || id != ent.ctx_id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    ent.addr = p;
+    // the lookup makes the device's context current if it was not: ask again for its id
+    ent.ctx_id = id ? id : current_context_id();
   }
-  *out = g_scratch_addr[dev];
+  *out = ent.addr;
   return cudaSuccess;
 }
 
@@ -47,11 +83,13 @@ cudaError_t scratch_address(void** out) {
 
 extern "C" pisa_status pisa_precompute_noalloc(const pisa_shape* shape, const void* q, const void* k, const void* v,
                                                const pisa_stats* stats, pisa_stream_t stream) {
+  // every check pisa_precompute makes (apart from its workspace) comes first: a rejected call
+  // enqueues nothing and leaves the shared scratch alone
+  pisa::Dims g;
+  const pisa_status s = pisa::validate_precompute(shape, q, k, v, stats, &g);
+  if (s != PISA_OK) return s;
   const size_t need = pisa_workspace_bytes(shape);
-  if (need == 0) {
-    // same validation as pisa_precompute, which reports the precise status
-    return pisa_precompute(shape, q, k, v, stats, nullptr, 0, stream);
-  }
+  if (need == 0) return PISA_ERR_INVALID_ARG;
   if (need > pisa::kNoAllocScratchBytes) return PISA_ERR_UNSUPPORTED;
   void* ws = nullptr;
   if (pisa::scratch_address(&ws) != cudaSuccess) return PISA_ERR_CUDA;

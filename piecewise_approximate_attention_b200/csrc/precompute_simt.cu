@@ -64,7 +64,8 @@ __device__ void block_moments(const T* q, const T* k, const T* v, int j, int L, 
   __syncthreads();
 }
 
-template <typename T, int D>
+// kFirstOrder = false: the zeroth-order statistics only (no partial sums of H_j).
+template <typename T, int D, bool kFirstOrder>
 __global__ void __launch_bounds__(kThreads) stats_partial(const T* __restrict__ q, const T* __restrict__ k,
                                                           const T* __restrict__ v, int L, int block, int nb,
                                                           pisa_stats st, float* __restrict__ partials) {
@@ -89,9 +90,10 @@ __global__ void __launch_bounds__(kThreads) stats_partial(const T* __restrict__ 
       st.vsum[so + c] = vb[c];
       st.qbar[so + c] = qb[c];
     }
-    accumulate_H<D>(Ks, Vs, block_count(j, L, block), acc);
+    if (kFirstOrder) accumulate_H<D>(Ks, Vs, block_count(j, L, block), acc);
     __syncthreads();
   }
+  if (!kFirstOrder) return;
   constexpr int kStep = kThreads / D;
   const int a0 = threadIdx.x / D, c = threadIdx.x % D;
   float* out = partials + ((size_t)bh * nparts + part) * D * D;
@@ -167,17 +169,24 @@ __global__ void __launch_bounds__(kThreads) cov_norm(const T* __restrict__ k, co
 
 template <typename T, int D>
 cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, const pisa_stats& st, void* ws,
-                cudaStream_t stream) {
+                bool first_order, cudaStream_t stream) {
   const int nparts = num_parts(g);
   float* partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
   const size_t smem_a = ((size_t)2 * g.block * D + 3 * D) * sizeof(float);
   const size_t smem_c = ((size_t)2 * g.block * D + 3 * D + kThreads / 32) * sizeof(float);
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(stats_partial<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a)))
+  if ((e = cudaFuncSetAttribute(stats_partial<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a)))
+    return e;
+  if ((e = cudaFuncSetAttribute(stats_partial<T, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a)))
     return e;
   if ((e = cudaFuncSetAttribute(cov_norm<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c)))
     return e;
-  stats_partial<T, D><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(
+  if (!first_order) {
+    stats_partial<T, D, false><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g.L, g.block, g.nb, st, partials);
+    return cudaGetLastError();
+  }
+  stats_partial<T, D, true><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g.L, g.block, g.nb, st, partials);
   hbar_reduce<D><<<dim3((D * D + kThreads - 1) / kThreads, g.BH()), kThreads, 0, stream>>>(
       partials, nparts, g.nb, g.scale, st.hbar, static_cast<__nv_bfloat16*>(st.hbar_op), nullptr, nullptr);
@@ -201,12 +210,13 @@ cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts,
 }
 
 cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,
-                                   const pisa_stats& st, void* ws, cudaStream_t stream) {
+                                   const pisa_stats& st, void* ws, bool first_order, cudaStream_t stream) {
   if (g.dtype == PISA_FP32) {
-    return g.d == 64 ? run<float, 64>(g, q, k, v, st, ws, stream) : run<float, 128>(g, q, k, v, st, ws, stream);
+    return g.d == 64 ? run<float, 64>(g, q, k, v, st, ws, first_order, stream)
+                     : run<float, 128>(g, q, k, v, st, ws, first_order, stream);
   }
-  return g.d == 64 ? run<__nv_bfloat16, 64>(g, q, k, v, st, ws, stream)
-                   : run<__nv_bfloat16, 128>(g, q, k, v, st, ws, stream);
+  return g.d == 64 ? run<__nv_bfloat16, 64>(g, q, k, v, st, ws, first_order, stream)
+                   : run<__nv_bfloat16, 128>(g, q, k, v, st, ws, first_order, stream);
 }
 
 }  // namespace pisa

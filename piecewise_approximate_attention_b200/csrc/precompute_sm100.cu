@@ -114,6 +114,11 @@ struct alignas(1024) SmemA {
   int abort;
 };
 
+// kFirstOrder: also accumulate the group's partial sum of H_j (tensor core) for Hbar.  Without it
+// (the zeroth-order pre-computation) the CTA writes the fp16 value operand with scale 1 from the V
+// tiles it streams, on the chance that the head's value scale is 1; value_scale_finish rewrites it
+// when it is not.
+template <bool kFirstOrder>
 __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_constant__ KVMaps maps, const PreParams p) {
   extern __shared__ uint8_t smem_raw[];
   SmemA& sm = *reinterpret_cast<SmemA*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -127,20 +132,20 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 129);
+      mbar_init(&sm.empty[s], kFirstOrder ? 129 : 128);   // the 128 column-sum threads (+ the MMA commit)
     }
     mbar_init(&sm.acc_done, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (kFirstOrder && warp == 5) {
     tmem_alloc(&sm.tmem_base, 128);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
+  const uint32_t tmem = kFirstOrder ? sm.tmem_base : 0u;
 
   if (warp == 4) {
     if (lane == 0) {
@@ -160,13 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
         ++issued;
       }
       {   // let issued copies land before shared memory is released (normally already landed)
-        const uint64_t t0 = globaltimer_ns();
-        for (int t = max(0, issued - 2); t < issued; ++t)
-          while (!mbar_try_wait(&sm.full[t & 1], (t >> 1) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+        for (int t = max(0, issued - 2); t < issued; ++t) mbar_drain(&sm.full[t & 1], (t >> 1) & 1, p.wait_ns);
       }
     }
   } else if (warp == 5) {
-    if (lane == 0) {
+    if (kFirstOrder && lane == 0) {
       bool ok = true;
       for (int t = 0; t < ntile && ok; ++t) {
         const int s = t & 1;
@@ -186,9 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
   } else {
     // column sums + rank-1 centring terms (threads 0..127)
     const int tid = threadIdx.x, cc = tid & 15, rg = tid >> 4;
-    float corr[D];
+    float corr[kFirstOrder ? D : 1];
 #pragma unroll
-    for (int c = 0; c < D; ++c) corr[c] = 0.f;
+    for (int c = 0; c < (kFirstOrder ? D : 1); ++c) corr[c] = 0.f;
     bool ok = true;
     int nblk = 0;
     float vabs = 0.f;
@@ -239,14 +242,37 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
         p.st.kbar[so] = sk * inv;
         p.st.vsum[so] = sv;
         reinterpret_cast<__nv_bfloat16*>(p.st.kbar_op)[so] = __float2bfloat16_rn(sk * inv);
-        const int pb = nblk & 1;
-        sm.ck[pb][c] = sk * inv;
-        sm.cv[pb][c] = sv;
-        bar_epi();
-        const float ka = sm.ck[pb][tid];
+        if constexpr (kFirstOrder) {
+          const int pb = nblk & 1;
+          sm.ck[pb][c] = sk * inv;
+          sm.cv[pb][c] = sv;
+          bar_epi();     // also: every thread has read red[] before the next block writes it
+          const float ka = sm.ck[pb][tid];
 #pragma unroll
-        for (int x = 0; x < D; ++x) corr[x] = fmaf(ka, sm.cv[pb][x], corr[x]);
+          for (int x = 0; x < D; ++x) corr[x] = fmaf(ka, sm.cv[pb][x], corr[x]);
+        } else {
+          bar_epi();     // every thread has read red[] before the next block writes it
+        }
         ++nblk;
+      }
+      if constexpr (!kFirstOrder) {
+        // fp16 value operand with scale 1 (exact for every bf16 value in fp16's range): 16-byte
+        // chunks of the swizzled V tile, consecutive chunks per thread
+        __half* vop = reinterpret_cast<__half*>(p.st.v_op) + (size_t)bh * p.L * D;
+        const int rbase = row0 + t * 128;
+        for (int q = tid; q < 128 * 16; q += 128) {
+          const int row = q >> 4, c = q & 15;
+          if (rbase + row >= row1) break;
+          const uint4 u = *reinterpret_cast<const uint4*>(sm.v[s] + (c >> 3) * kHalf + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          uint32_t hw[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const __half2 h2 = __floats2half2_rn(__uint_as_float(w[x] << 16), __uint_as_float(w[x] & 0xffff0000u));
+            hw[x] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          *reinterpret_cast<uint4*>(vop + (size_t)(rbase + row) * D + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
       }
       mbar_arrive(&sm.empty[s]);
     }
@@ -256,34 +282,72 @@ __global__ void __launch_bounds__(kThreads, 1) stats_a_sm100(const __grid_consta
     bar_epi();
     if (tid == 0)
       p.vmax[(size_t)bh * nparts + part] = fmaxf(fmaxf(sm.red[0][0][0], sm.red[0][0][1]), fmaxf(sm.red[0][0][2], sm.red[0][0][3]));
-    if (ok) ok = !epi_any_failed(!wait_bar(&sm.acc_done, 0, &sm.abort, p.status, p.wait_ns));
-    if (ok) {
-      tc_fence_after();
-      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-      float* out = p.partials + ((size_t)bh * nparts + part) * D * D + (size_t)tid * D;
+    if constexpr (kFirstOrder) {
+      if (ok) ok = !epi_any_failed(!wait_bar(&sm.acc_done, 0, &sm.abort, p.status, p.wait_ns));
+      if (ok) {
+        tc_fence_after();
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        float* out = p.partials + ((size_t)bh * nparts + part) * D * D + (size_t)tid * D;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        float a[32];
-        tmem_ld32(trow + 32 * ch, a);
-        tmem_ld_wait();
-        if (ntile == 0) {
+        for (int ch = 0; ch < 4; ++ch) {
+          float a[32];
+          tmem_ld32(trow + 32 * ch, a);
+          tmem_ld_wait();
+          if (ntile == 0) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) a[x] = 0.f;
+            for (int x = 0; x < 32; ++x) a[x] = 0.f;
+          }
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(out + 32 * ch + x) =
+                make_float4(a[x] - corr[32 * ch + x], a[x + 1] - corr[32 * ch + x + 1], a[x + 2] - corr[32 * ch + x + 2],
+                            a[x + 3] - corr[32 * ch + x + 3]);
         }
-#pragma unroll
-        for (int x = 0; x < 32; x += 4)
-          *reinterpret_cast<float4*>(out + 32 * ch + x) =
-              make_float4(a[x] - corr[32 * ch + x], a[x + 1] - corr[32 * ch + x + 1], a[x + 2] - corr[32 * ch + x + 2],
-                          a[x + 3] - corr[32 * ch + x + 3]);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (kFirstOrder && warp == 5) {
     __syncwarp();
     tmem_dealloc(tmem, 128);
+  }
+}
+
+// Zeroth-order pre-computation, second launch: one CTA per (head, group of kBlocksPerPart key
+// blocks).  Every CTA of a head derives the head's value scale from the groups' max |v| (the same
+// rule as hbar_reduce: the smallest power of two >= max|v| / 256); the first writes it.  Each CTA
+// writes its blocks' fp16 value sums vsum / vscale and, when the scale is not 1, rewrites its rows
+// of the fp16 value operand (stats_a_sm100<false> wrote them with scale 1).
+__global__ void __launch_bounds__(256) value_scale_finish(const __nv_bfloat16* __restrict__ v, const PreParams p) {
+  const int part = blockIdx.x, bh = blockIdx.y, nparts = gridDim.x;
+  float mx = 0.f;
+  for (int i = 0; i < nparts; ++i) mx = fmaxf(mx, p.vmax[(size_t)bh * nparts + i]);
+  float sc = 1.f;
+  while (mx > 256.f * sc && sc < 0x1p100f) sc *= 2.f;
+  if (part == 0 && threadIdx.x == 0) p.st.vscale[bh] = sc;
+  const float vinv = 1.f / sc;
+  const int jb0 = part * kBlocksPerPart, jb1 = min(p.nb, jb0 + kBlocksPerPart);
+  __half* vsop = reinterpret_cast<__half*>(p.st.vsum_op);
+  for (int e = threadIdx.x; e < (jb1 - jb0) * D; e += blockDim.x) {
+    const size_t so = ((size_t)bh * p.nb + jb0) * D + e;
+    vsop[so] = __float2half_rn(p.st.vsum[so] * vinv);
+  }
+  if (sc == 1.f) return;
+  const int row0 = jb0 * p.block, row1 = min(p.L, jb1 * p.block);
+  const uint4* src = reinterpret_cast<const uint4*>(v + (size_t)bh * p.L * D);
+  uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p.st.v_op) + (size_t)bh * p.L * D);
+  for (size_t e = (size_t)row0 * (D / 8) + threadIdx.x; e < (size_t)row1 * (D / 8); e += blockDim.x) {
+    const uint4 u = src[e];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t hw[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const __half2 h2 = __floats2half2_rn(__uint_as_float(w[x] << 16) * vinv, __uint_as_float(w[x] & 0xffff0000u) * vinv);
+      hw[x] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    dst[e] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
   }
 }
 
@@ -358,9 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
         ++issued;
       }
       {   // let issued copies land before shared memory is released (normally already landed)
-        const uint64_t t0 = globaltimer_ns();
         for (int t = max(0, issued - kStagesB); t < issued; ++t)
-          while (!mbar_try_wait(&sm.full[t % kStagesB], (t / kStagesB) & 1) && globaltimer_ns() - t0 < p.wait_ns) {}
+          mbar_drain(&sm.full[t % kStagesB], (t / kStagesB) & 1, p.wait_ns);
       }
     }
   } else if (warp == 5) {
@@ -506,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) cov_norm_sm100(const __grid_const
 }  // namespace
 
 cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v, const pisa_stats& st,
-                                    void* ws, cudaStream_t stream) {
+                                    void* ws, bool first_order, cudaStream_t stream) {
   KVMaps maps;
   const uint64_t bh = (uint64_t)g.BH();
   if (!encode_bf16_3d(&maps.q, q, D, g.L, bh, 128) || !encode_bf16_3d(&maps.k, k, D, g.L, bh, 128) ||
@@ -524,11 +587,17 @@ cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k,
   p.wait_ns = kWaitLimitNs;
   const size_t smem_a = sizeof(SmemA) + 1024, smem_b = sizeof(SmemB) + 1024;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(stats_a_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
+  if ((e = cudaFuncSetAttribute(stats_a_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
+  if ((e = cudaFuncSetAttribute(stats_a_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
   if ((e = cudaFuncSetAttribute(cov_norm_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
   if ((e = cudaFuncSetAttribute(cov_norm_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
   const int nparts = num_parts(g);
-  stats_a_sm100<<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(maps, p);
+  if (!first_order) {
+    stats_a_sm100<false><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(maps, p);
+    value_scale_finish<<<dim3(nparts, g.BH()), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(v), p);
+    return cudaGetLastError();
+  }
+  stats_a_sm100<true><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(maps, p);
   if ((e = launch_hbar_reduce(g, p.partials, nparts, p.vmax, st, stream))) return e;
   const dim3 grid_b((g.nb + kBlocksPerCtaB - 1) / kBlocksPerCtaB, g.BH());
   if (st.hdiff_op)

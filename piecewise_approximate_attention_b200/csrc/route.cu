@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const float* __restr
   const int bh = blockIdx.y, i0 = blockIdx.x * kRows;
   const int rows = min(kRows, nb - i0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* Mh = M + (size_t)bh * nb;
+  const float* Mh = M ? M + (size_t)bh * nb : nullptr;    // null: lambda == 0, the M term is dropped
 
   static_assert(kRows * D % kThreads == 0, "query rows per thread");
 #pragma unroll
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const float* __restr
   float msum = 0.f;
 #pragma unroll 4
   for (int j = threadIdx.x; j < nb; j += kThreads) {
-    const float mv = Mh[j];
+    const float mv = Mh ? Mh[j] : 0.f;
     Ms[j] = mv;
     msum += mv;
   }
@@ -325,8 +325,9 @@ cudaError_t launch_route_kernel(const Dims& g, const pisa_stats& st, int keep_k,
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(route_kernel<D, kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
     return e;
+  // lambda == 0 drops the M term: M is not read (it may be unwritten)
   route_kernel<D, kRows><<<dim3((g.nb + kRows - 1) / kRows, g.BH()), kThreads, smem, stream>>>(
-      st.qbar, st.kbar, st.M, g.L, g.block, g.nb, g.scale, keep_k, lam, sel, scores);
+      st.qbar, st.kbar, lam > 0.f ? st.M : nullptr, g.L, g.block, g.nb, g.scale, keep_k, lam, sel, scores);
   return cudaGetLastError();
 }
 

@@ -14,13 +14,19 @@ class Pisa:
     """Reusable PISA attention for a fixed [B, H, L, d] shape, block size, keep_k and lambda.
 
     ``pair=True`` asks the router for the query-block pairing order used by 128-row tiles when
-    block == 64 (a scheduling choice: the output does not depend on it).
+    block == 64 (a scheduling choice: the output does not depend on it).  ``first_order=False``
+    makes ``precompute`` write the zeroth-order statistics only (pisa_precompute_zeroth_order):
+    enough for lambda = 0 routing and the keep-or-drop mode, i.e. an exact-only pipeline.
     """
 
     def __init__(self, batch: int, heads: int, seq_len: int, head_dim: int, block: int, keep_k: int,
                  lam: float, dtype: str = "bf16", softmax_scale: float = 1.0, device="cuda",
-                 mode: int = C.PISA_MODE_PISA, with_H: bool = False, pair: bool = True):
+                 mode: int = C.PISA_MODE_PISA, with_H: bool = False, pair: bool = True,
+                 first_order: bool = True):
         import torch
+        if not first_order and (lam != 0.0 or mode != C.PISA_MODE_EXACT_ONLY):
+            raise ValueError("the zeroth-order statistics serve lambda = 0 routing and PISA_MODE_EXACT_ONLY only")
+        self.first_order = first_order
         self.shape = C.make_shape(batch, heads, seq_len, head_dim, block, dtype, softmax_scale)
         self.block, self.keep_k, self.lam, self.mode = block, keep_k, lam, mode
         self.nb = C.pisa_num_blocks(seq_len, block)
@@ -36,7 +42,10 @@ class Pisa:
         self.order = torch.empty((batch, heads, self.nb), dtype=torch.int32, device=self.device) if pair else None
 
     def precompute(self, q, k, v, stream=None):
-        C.pisa_precompute(self.shape, q, k, v, self.stats, self.ws, stream)
+        if self.first_order:
+            C.pisa_precompute(self.shape, q, k, v, self.stats, self.ws, stream)
+        else:
+            C.pisa_precompute_zeroth_order(self.shape, q, k, v, self.stats, self.ws, stream)
 
     def route(self, scores=None, stream=None):
         C.pisa_route(self.shape, self.stats, self.keep_k, self.lam, self.sel, self.order, scores, stream)
@@ -75,11 +84,13 @@ class Pisa:
         return graph
 
     def launches_per_step(self) -> int:
-        """Kernels one __call__ enqueues: pre-compute 3 (+3 e4m3 quantizations), routing 1 (+1
-        pairing), attention 1 (+1 for the per-block first-order kernel on the bf16 path)."""
+        """Kernels one __call__ enqueues: pre-compute 3 (2 zeroth-order only on the bf16 path, 1 on
+        the fp32 path; +3 e4m3 quantizations), routing 1 (+1 pairing), attention 1 (+1 for the
+        per-block first-order kernel on the bf16 path)."""
         extra = 1 if (self.mode == C.PISA_MODE_PER_BLOCK and self.tdtype != self._torch_f32 and
                       self.keep_k < self.nb) else 0
-        return 3 + (3 if self.fp8 else 0) + 1 + (1 if self.order is not None else 0) + 1 + extra
+        pre = 3 if self.first_order else (1 if self.tdtype == self._torch_f32 else 2)
+        return pre + (3 if self.fp8 else 0) + 1 + (1 if self.order is not None else 0) + 1 + extra
 
     def device_error(self, stream=None):
         return C.pisa_read_device_error(self.ws, stream)

@@ -136,15 +136,29 @@ def make_qkv(w: Workload, heads: Optional[Sequence[int]] = None, seed: Optional[
     ``heads`` selects a subset of the workload's heads (default: all); head h always gets the same
     values whatever subset it is drawn in, so sampled checks see the full-size run's inputs.
     """
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
     import torch
     hs = list(range(w.heads)) if heads is None else list(heads)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     L, d = w.seq_len, w.head_dim
     out = [torch.empty((w.batch, len(hs), L, d), dtype=tdt) for _ in range(3)]
-    for b in range(w.batch):
-        for i, h in enumerate(hs):
-            for t, arr in zip(out, make_head(w, b, h, seed)):
-                t[b, i].copy_(to_dtype(arr, w.dtype))
+
+    def fill(bi):
+        b, i = bi
+        for t, arr in zip(out, make_head(w, b, hs[i], seed)):
+            t[b, i].copy_(to_dtype(arr, w.dtype))
+
+    # every (batch, head) draws from its own stream, so filling them on threads gives the same values
+    jobs = [(b, i) for b in range(w.batch) for i in range(len(hs))]
+    workers = min(len(jobs), os.cpu_count() or 1, 16)
+    if workers <= 1:
+        for job in jobs:
+            fill(job)
+    else:
+        with ThreadPoolExecutor(workers) as ex:
+            list(ex.map(fill, jobs))
     return out[0], out[1], out[2]
 
 

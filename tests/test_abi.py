@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_blocks():
-    assert C.lib().pisa_abi_version() == 5
+    assert C.lib().pisa_abi_version() == 6
     assert C.pisa_num_blocks(32760, 64) == 512
     assert C.pisa_num_blocks(75600, 128) == 591
     assert C.pisa_num_blocks(1, 64) == 1
@@ -107,6 +107,8 @@ def test_bad_shapes_rejected(kw, expect):
     sh = _shape(**kw)
     st = C.PisaStats()
     assert C.lib().pisa_precompute(ctypes.byref(sh), 16, 16, 16, ctypes.byref(st), 16, 1 << 30, None) == expect
+    assert C.lib().pisa_precompute_zeroth_order(ctypes.byref(sh), 16, 16, 16, ctypes.byref(st), 16, 1 << 30,
+                                                None) == expect
     assert C.pisa_stats_bytes(sh, False) == 0
     assert C.pisa_workspace_bytes(sh) == 0
     assert C.pisa_perblock_workspace_bytes(sh) == 0
@@ -133,6 +135,13 @@ def test_invalid_arguments_rejected_without_launch():
     bad = C.PisaStats.from_buffer_copy(st)
     bad.kbar_op = None
     assert L.pisa_precompute(bs, P, P, P, ctypes.byref(bad), P, ws, None) == C.PISA_ERR_INVALID_ARG
+    # the zeroth-order pre-computation checks the same arguments
+    Z = L.pisa_precompute_zeroth_order
+    assert Z(bs, None, P, P, ctypes.byref(st), P, ws, None) == C.PISA_ERR_INVALID_ARG
+    assert Z(bs, P + 4, P, P, ctypes.byref(st), P, ws, None) == C.PISA_ERR_INVALID_ARG
+    assert Z(bs, P, P, P, ctypes.byref(st), P, ws - 1, None) == C.PISA_ERR_INVALID_ARG
+    assert Z(bs, P, P, P, ctypes.byref(st), None, ws, None) == C.PISA_ERR_INVALID_ARG
+    assert Z(bs, P, P, P, ctypes.byref(bad), P, ws, None) == C.PISA_ERR_INVALID_ARG
     # routing arguments
     assert L.pisa_route(bs, ctypes.byref(st), 17, 0.5, P, None, None, None) == C.PISA_ERR_INVALID_ARG
     assert L.pisa_route(bs, ctypes.byref(st), -1, 0.5, P, None, None, None) == C.PISA_ERR_INVALID_ARG
@@ -225,4 +234,4 @@ def test_headers_are_plain_c_and_the_library_links_from_c(tmp_path):
                     f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
     res = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0, res.stderr
-    assert "c consumer ok: abi 5" in res.stdout
+    assert "c consumer ok: abi 6" in res.stdout

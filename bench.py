@@ -249,13 +249,21 @@ def run_ours(args, rank, world, local_rank):
         o = torch.empty_like(qd)
     torch.cuda.synchronize()
 
+    fused = p.fused_short_step()
+
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        p.precompute(qd, kd, vd, stream)
-        if evs:
-            evs[1].record(stream)
-        p.route(stream=stream)
+        if fused:
+            # short sequences: pre-computation and routing in one cluster launch (timed as pre-compute)
+            p.precompute_route(qd, kd, vd, stream=stream)
+            if evs:
+                evs[1].record(stream)
+        else:
+            p.precompute(qd, kd, vd, stream)
+            if evs:
+                evs[1].record(stream)
+            p.route(stream=stream)
         if evs:
             evs[2].record(stream)
         p.attention(qd, kd, vd, o, stream=stream)
@@ -573,9 +581,10 @@ SHORT_WORKLOADS = ("image-dit", "sweep-L8192-s0.875")
 
 def short_sequences(dev, reps: int = 30):
     """Short sequences, where per-launch overhead and the pre-computation weigh most: the full
-    step (pre-compute + route + attention) launched call by call and replayed as one CUDA graph,
-    its parts, and the library's dense attention on the same inputs, timed interleaved (medians).
-    Outside the timed region."""
+    step (pre-compute and route in one cluster launch + attention) launched call by call and
+    replayed as one CUDA graph, its parts (the fused pre-compute + route, and the separate
+    pre-compute and route calls), and the library's dense attention on the same inputs, timed
+    interleaved (medians).  Outside the timed region."""
     import torch
     from piecewise_approximate_attention_b200.runtime import Pisa
     from piecewise_approximate_attention_b200.workloads import WORKLOADS, make_qkv
@@ -588,10 +597,13 @@ def short_sequences(dev, reps: int = 30):
         p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, dev)
         o = torch.empty_like(q)
         graph = p.capture(q, k, v, o)
+        graph_sep = p.capture(q, k, v, o, fused=False)
         dense = Pisa(B, H, L, d, w.block, p.nb, w.lam, w.dtype, 1.0, dev, pair=False)
         dense.precompute(q, k, v)
         dense.route()
         arms = {"step_launches": lambda: p(q, k, v, o), "step_graph": graph.replay,
+                "step_graph_separate_precompute_route": graph_sep.replay,
+                "precompute_route_fused": lambda: p.precompute_route(q, k, v),
                 "precompute": lambda: p.precompute(q, k, v), "route": lambda: p.route(),
                 "attention": lambda: p.attention(q, k, v, o), "dense_attention": lambda: dense.attention(q, k, v, o)}
         with NvmlClock(dev.index or 0) as nclk:
@@ -602,7 +614,7 @@ def short_sequences(dev, reps: int = 30):
                      "p10_p90_ms_step_graph": [st["step_graph"]["p10_ms"], st["step_graph"]["p90_ms"]],
                      "sm_mhz": st["step_graph"]["sm_mhz"],
                      "speedup_step_vs_dense": round(st["dense_attention"]["median_ms"] / st["step_graph"]["median_ms"], 3)}
-        del graph, p, dense
+        del graph, graph_sep, p, dense
     return out
 
 
@@ -746,7 +758,12 @@ def profile_case(a):
         o_r = torch.empty_like(q)
     for _ in range(a.iters):
         if perm is None:
-            p(q, k, v, o)
+            if a.fused:
+                p.precompute_route(q, k, v)
+            else:
+                p.precompute(q, k, v)
+                p.route()
+            p.attention(q, k, v, o)
         else:
             for x, b in zip((q, k, v), bufs):
                 reorder_tokens(x, perm, out=b)
@@ -778,6 +795,8 @@ def main():
     ap.add_argument("--mode", choices=("pisa", "per_block"), default="pisa")
     ap.add_argument("--dtype", choices=("bf16", "bf16_fp8qk"), default="bf16")
     ap.add_argument("--reorder", default=None, help="axis order of the frames x height x width grid, e.g. hwt")
+    ap.add_argument("--fused", action="store_true", help="profile case: pre-compute and route through "
+                    "pisa_precompute_route (one cluster launch for short sequences)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

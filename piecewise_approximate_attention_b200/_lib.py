@@ -21,7 +21,7 @@ PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
            "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string",
            "pisa_precompute_noalloc", "pisa_testing_set_attention_fault", "pisa_perblock_workspace_bytes",
-           "pisa_permute_rows", "pisa_axis_permutation", "pisa_precompute_zeroth_order")
+           "pisa_permute_rows", "pisa_axis_permutation", "pisa_precompute_zeroth_order", "pisa_precompute_route")
 
 
 class PisaShape(ctypes.Structure):
@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
             "pisa_precompute": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, sz, vp]),
             "pisa_precompute_zeroth_order": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, sz, vp]),
             "pisa_route": (i32, [P(PisaShape), P(PisaStats), i32, f32, vp, vp, vp, vp]),
+            "pisa_precompute_route": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), i32, f32, vp, vp, vp, vp, sz,
+                                            vp]),
             "pisa_attention": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, vp, i32, i32, vp, vp, sz, vp]),
             "pisa_read_device_error": (i32, [vp, P(i32), vp]),
             "pisa_status_string": (ctypes.c_char_p, [i32]),
@@ -219,6 +221,14 @@ def pisa_precompute_noalloc(shape: PisaShape, q, k, v, stats: Stats, stream=None
 def pisa_route(shape: PisaShape, stats: Stats, keep_k: int, lam: float, sel, order=None, scores=None, stream=None):
     _check(lib().pisa_route(ctypes.byref(shape), ctypes.byref(stats.c), int(keep_k), float(lam), _ptr(sel),
                             _ptr(order), _ptr(scores), _stream(stream)), "pisa_route")
+
+
+def pisa_precompute_route(shape: PisaShape, q, k, v, stats: Stats, keep_k: int, lam: float, sel, order, scores, ws,
+                          stream=None):
+    """pisa_precompute then pisa_route; one cluster launch for bf16 inputs with nb <= 128."""
+    _check(lib().pisa_precompute_route(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(stats.c),
+                                       int(keep_k), float(lam), _ptr(sel), _ptr(order), _ptr(scores), _ptr(ws),
+                                       ws.numel(), _stream(stream)), "pisa_precompute_route")
 
 
 def pisa_attention(shape: PisaShape, q, k, v, stats: Stats, sel, order, keep_k: int, mode: int, o, ws, stream=None):

@@ -204,17 +204,45 @@ pisa_status pisa_precompute_zeroth_order(const pisa_shape* shape, const void* q,
   return precompute(shape, q, k, v, stats, ws, ws_bytes, false, stream);
 }
 
+namespace {
+pisa_status check_route_args(const Dims& g, int32_t keep_k, float lambda, const int32_t* sel, const int32_t* order,
+                             const float* scores) {
+  if (keep_k < 0 || keep_k > g.nb || !std::isfinite(lambda) || lambda < 0.f) return PISA_ERR_INVALID_ARG;
+  if ((keep_k > 0 && (!sel || !aligned16(sel))) || (order && !aligned16(order)) || (scores && !aligned16(scores)))
+    return PISA_ERR_INVALID_ARG;
+  return PISA_OK;
+}
+}  // namespace
+
 pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,
                        int32_t* sel, int32_t* order, float* scores, pisa_stream_t stream) {
   Dims g;
   pisa_status s = check_shape(shape, &g);
   if (s != PISA_OK) return s;
   if ((s = check_stats(g, stats, false)) != PISA_OK) return s;
-  if (keep_k < 0 || keep_k > g.nb || !std::isfinite(lambda) || lambda < 0.f) return PISA_ERR_INVALID_ARG;
-  if ((keep_k > 0 && (!sel || !aligned16(sel))) || (order && !aligned16(order)) || (scores && !aligned16(scores)))
-    return PISA_ERR_INVALID_ARG;
+  if ((s = check_route_args(g, keep_k, lambda, sel, order, scores)) != PISA_OK) return s;
   return cuda_status(launch_route(g, *stats, keep_k, lambda, sel, order, scores,
                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+pisa_status pisa_precompute_route(const pisa_shape* shape, const void* q, const void* k, const void* v,
+                                  const pisa_stats* stats, int32_t keep_k, float lambda, int32_t* sel,
+                                  int32_t* order, float* scores, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+  Dims g;
+  pisa_status s = validate_precompute(shape, q, k, v, stats, &g);
+  if (s != PISA_OK) return s;
+  if (!ws || !aligned16(ws) || ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
+  if ((s = check_route_args(g, keep_k, lambda, sel, order, scores)) != PISA_OK) return s;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  bool launched = false;
+  cudaError_t e = launch_short_step_sm100(g, q, k, v, *stats, ws, keep_k, lambda, sel, order, scores, cs, &launched);
+  if (e != cudaSuccess) return PISA_ERR_CUDA;
+  if (launched) {
+    if (g.dtype == PISA_BF16_FP8QK) e = launch_quantize_fp8(g, q, k, *stats, cs);
+    return cuda_status(e);
+  }
+  if ((s = pisa_precompute(shape, q, k, v, stats, ws, ws_bytes, stream)) != PISA_OK) return s;
+  return pisa_route(shape, stats, keep_k, lambda, sel, order, scores, stream);
 }
 
 pisa_status pisa_attention(const pisa_shape* shape, const void* q, const void* k, const void* v,

@@ -99,6 +99,13 @@ cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts,
                                const pisa_stats& st, cudaStream_t stream);
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream);
+// Pre-computation + routing in one cluster launch (bf16 inputs, d = 128, nb <= 128).  *launched is
+// false (and nothing is enqueued) when the shape is not eligible or the device cannot schedule the
+// cluster; the caller then runs the separate kernels.
+bool short_step_eligible(const Dims& g);
+cudaError_t launch_short_step_sm100(const Dims& g, const void* q, const void* k, const void* v, const pisa_stats& st,
+                                    void* ws, int keep_k, float lam, int32_t* sel, int32_t* order, float* scores,
+                                    cudaStream_t stream, bool* launched);
 cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const int32_t* sel, const int32_t* order,
                                    int keep_k, int mode, const float* vscale, const F8Scales& f8, void* o,
                                    float2* rowstats, float* o32, int* status, unsigned long long wait_ns, int fault,

@@ -47,6 +47,19 @@ class Pisa:
         else:
             C.pisa_precompute_zeroth_order(self.shape, q, k, v, self.stats, self.ws, stream)
 
+    def fused_short_step(self) -> bool:
+        """Whether precompute_route runs as one cluster launch (bf16 inputs, head_dim 128, nb <= 128)."""
+        return self.first_order and self.tdtype != self._torch_f32 and self.shape.head_dim == 128 and self.nb <= 128
+
+    def precompute_route(self, q, k, v, scores=None, stream=None):
+        """Pre-computation and routing; for short sequences one cluster launch (same results)."""
+        if not self.first_order:
+            self.precompute(q, k, v, stream)
+            self.route(scores, stream)
+            return
+        C.pisa_precompute_route(self.shape, q, k, v, self.stats, self.keep_k, self.lam, self.sel, self.order, scores,
+                                self.ws, stream)
+
     def route(self, scores=None, stream=None):
         C.pisa_route(self.shape, self.stats, self.keep_k, self.lam, self.sel, self.order, scores, stream)
 
@@ -60,16 +73,16 @@ class Pisa:
         import torch
         if o is None:
             o = torch.empty_like(q)
-        self.precompute(q, k, v, stream)
-        self.route(stream=stream)
+        self.precompute_route(q, k, v, stream=stream)
         self.attention(q, k, v, o, stream=stream)
         return o
 
-    def capture(self, q, k, v, o):
+    def capture(self, q, k, v, o, fused: bool = True):
         """Records one full step (pre-computation, routing, attention of q, k, v into o) as a CUDA
         graph and returns it; ``graph.replay()`` then re-runs the step on whatever the same
         buffers hold, with one launch from the host.  The buffers must stay allocated while the
-        graph is used.  The step runs once eagerly first (outside the capture)."""
+        graph is used.  The step runs once eagerly first (outside the capture).  ``fused=False``
+        records the separate pre-computation and routing calls instead of precompute_route."""
         import torch
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
@@ -78,19 +91,26 @@ class Pisa:
         torch.cuda.current_stream(self.device).wait_stream(side)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side):
-            self.precompute(q, k, v)
-            self.route()
+            if fused:
+                self.precompute_route(q, k, v)
+            else:
+                self.precompute(q, k, v)
+                self.route()
             self.attention(q, k, v, o)
         return graph
 
     def launches_per_step(self) -> int:
         """Kernels one __call__ enqueues: pre-compute 3 (2 zeroth-order only on the bf16 path, 1 on
-        the fp32 path; +3 e4m3 quantizations), routing 1 (+1 pairing), attention 1 (+1 for the
+        the fp32 path; +3 e4m3 quantizations), routing 1 (+1 pairing) -- or, for short bf16
+        sequences, pre-compute and routing in 1 cluster launch -- and attention 1 (+1 for the
         per-block first-order kernel on the bf16 path)."""
         extra = 1 if (self.mode == C.PISA_MODE_PER_BLOCK and self.tdtype != self._torch_f32 and
                       self.keep_k < self.nb) else 0
         pre = 3 if self.first_order else (1 if self.tdtype == self._torch_f32 else 2)
-        return pre + (3 if self.fp8 else 0) + 1 + (1 if self.order is not None else 0) + 1 + extra
+        route = 1 + (1 if self.order is not None else 0)
+        if self.fused_short_step():
+            pre, route = 1, 0          # pre-computation and routing in one cluster launch
+        return pre + (3 if self.fp8 else 0) + route + 1 + extra
 
     def device_error(self, stream=None):
         return C.pisa_read_device_error(self.ws, stream)

@@ -195,7 +195,7 @@ cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, cons
                 const int32_t* sel, int keep_k, int mode, void* o, int* status, cudaStream_t stream) {
   const size_t smem = sizeof(Smem<D>);
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(attn_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_simt<T, D>), smem))) return e;
   attn_simt<T, D><<<dim3(g.nb, g.BH()), g.block, smem, stream>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), st, sel, keep_k, mode, g.L,
       g.block, g.nb, g.scale, static_cast<T*>(o), status);

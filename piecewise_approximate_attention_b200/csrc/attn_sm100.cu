@@ -74,7 +74,6 @@ struct alignas(1024) Smem {
 
 struct Params {
   int L, nb, block, keep_k, mode, dense;
-  int rank_major;            // grid (heads, tiles) instead of (tiles, heads): see the launcher
   float scale_log2;
   float lazy;                // rescale O only when the row max grows by more than this (logit units)
   const float* vscale;       // [B*H] value scale of the fp16 value operands
@@ -169,7 +168,7 @@ attn_sm100(const __grid_constant__ AttnMaps maps, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = p.rank_major ? blockIdx.y : blockIdx.x, bh = p.rank_major ? blockIdx.x : blockIdx.y;
+  const int tile = blockIdx.x, bh = blockIdx.y;
   const bool pair = p.block == 64;
 
   // ---- query blocks of this tile ----
@@ -676,20 +675,12 @@ cudaError_t launch_attention_sm100(const Dims& g, const AttnMaps& maps, const in
   const size_t smem = attention_sm100_smem_bytes();
   cudaError_t e;
   const int ntiles = g.block == 64 ? (g.nb + 1) / 2 : g.nb;
-  // CTAs start in linear block order.  Tile costs differ only with pairing (block 64: the union of
-  // two selections), and the pairing order lists a head's pairs by decreasing union.  When every
-  // head's keys and values fit in L2 together (short sequences), the grid runs rank-major -- the
-  // first tile of every head, then the second, ... -- so the longest tiles start first and the last
-  // wave's tail is short.  Otherwise it stays head-major, which keeps the keys and values that
-  // neighbouring query tiles share in L2.
-  const double kv_bytes = (double)g.BH() * g.L * D * 4.0;     // bf16 keys + fp16 values
-  p.rank_major = (g.block == 64 && order != nullptr && kv_bytes <= 80e6) ? 1 : 0;
-  const dim3 grid = p.rank_major ? dim3(g.BH(), ntiles) : dim3(ntiles, g.BH());
+  const dim3 grid(ntiles, g.BH());
   if (f8.q) {
-    if ((e = cudaFuncSetAttribute(attn_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+    if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_sm100<true>), smem))) return e;
     attn_sm100<true><<<grid, kThreads, smem, stream>>>(maps, p);
   } else {
-    if ((e = cudaFuncSetAttribute(attn_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+    if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(attn_sm100<false>), smem))) return e;
     attn_sm100<false><<<grid, kThreads, smem, stream>>>(maps, p);
   }
   return cudaGetLastError();

@@ -84,6 +84,15 @@ bool encode_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t r
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // bounded mbarrier waits: 2 s
 
+// cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) on the current
+// device, made only when this kernel has not yet been given at least `bytes` there: the driver
+// call would otherwise be repeated, on the host, before every launch.
+cudaError_t set_max_dynamic_smem(const void* fn, size_t bytes);
+
+// Unique id of the calling thread's current CUDA context, 0 if none is current (or the driver
+// cannot say).  Host caches of per-context state key on it.
+unsigned long long current_context_id();
+
 // Argument checks of pisa_precompute other than its workspace (shape, q, k, v, stats); fills *g.
 // Enqueues nothing.  Shared by the entry points that run the pre-computation.
 pisa_status validate_precompute(const pisa_shape* shape, const void* q, const void* k, const void* v,

@@ -381,7 +381,7 @@ cudaError_t launch_perblock_sm100(const Dims& g, const AttnMaps& maps, const CUt
   p.wait_ns = wait_ns;
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(perblock_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))) return e;
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(perblock_sm100), smem))) return e;
   const int ntiles = g.block == 64 ? (g.nb + 1) / 2 : g.nb;
   perblock_sm100<<<dim3(ntiles, g.BH()), kThreads, smem, stream>>>(maps, hdiff, p);
   return cudaGetLastError();

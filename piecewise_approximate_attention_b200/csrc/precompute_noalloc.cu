@@ -11,8 +11,6 @@
 // host-side stand-in, so its device address is looked up with cudaGetSymbolAddress, with the device
 // current, the first time a call runs in a device's CUDA context (and again if that context has been
 // replaced, e.g. after cudaDeviceReset, since the module is then loaded afresh).
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 #include "common.cuh"
@@ -31,30 +29,6 @@ struct ScratchEntry {
   void* addr = nullptr;
 };
 ScratchEntry g_scratch[kMaxDevices];
-
-// Unique id of the calling thread's current CUDA context (0 if none is current or the driver
-// cannot say).  Driver entry points through the runtime: no link-time dependency on libcuda.
-unsigned long long current_context_id() {
-  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
-  static PFN_cuCtxGetId_v12000 get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
-  });
-  if (!get_cur || !get_id) return 0;
-  CUcontext ctx = nullptr;
-  unsigned long long id = 0;
-  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
-  return id;
-}
 
 // Device address of g_noalloc_scratch in the current device's context.  Looked up once per
 // context; a host-side query that allocates nothing.

@@ -175,11 +175,11 @@ cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, cons
   const size_t smem_a = ((size_t)2 * g.block * D + 3 * D) * sizeof(float);
   const size_t smem_c = ((size_t)2 * g.block * D + 3 * D + kThreads / 32) * sizeof(float);
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(stats_partial<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a)))
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(stats_partial<T, D, true>), smem_a)))
     return e;
-  if ((e = cudaFuncSetAttribute(stats_partial<T, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a)))
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(stats_partial<T, D, false>), smem_a)))
     return e;
-  if ((e = cudaFuncSetAttribute(cov_norm<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c)))
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(cov_norm<T, D>), smem_c)))
     return e;
   if (!first_order) {
     stats_partial<T, D, false><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(

@@ -121,10 +121,10 @@ cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k,
   p.wait_ns = kWaitLimitNs;
   const size_t smem_a = sizeof(SmemA) + 1024, smem_b = sizeof(SmemB) + 1024;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(stats_a_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
-  if ((e = cudaFuncSetAttribute(stats_a_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
-  if ((e = cudaFuncSetAttribute(cov_norm_sm100<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
-  if ((e = cudaFuncSetAttribute(cov_norm_sm100<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(stats_a_sm100<true>), smem_a))) return e;
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(stats_a_sm100<false>), smem_a))) return e;
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(cov_norm_sm100<false>), smem_b))) return e;
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(cov_norm_sm100<true>), smem_b))) return e;
   const int nparts = num_parts(g);
   if (!first_order) {
     stats_a_sm100<false><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(maps, p);

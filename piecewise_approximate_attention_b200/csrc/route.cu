@@ -44,7 +44,7 @@ cudaError_t launch_route_kernel(const Dims& g, const pisa_stats& st, int keep_k,
                                 float* scores, cudaStream_t stream) {
   const size_t smem = route_smem_floats<D, kRows>(g.nb) * sizeof(float);
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(route_kernel<D, kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(route_kernel<D, kRows>), smem)))
     return e;
   // lambda == 0 drops the M term: M is not read (it may be unwritten)
   route_kernel<D, kRows><<<dim3((g.nb + kRows - 1) / kRows, g.BH()), kRouteThreads, smem, stream>>>(
@@ -68,7 +68,7 @@ cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float 
   if (order) {
     if (g.block == 64 && keep_k > 0 && g.nb > 2) {
       const size_t psmem = pair_smem_bytes(g.nb);
-      if ((e = cudaFuncSetAttribute(pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem))) return e;
+      if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(pair_kernel), psmem))) return e;
       pair_kernel<<<dim3((g.nb + kSeg - 1) / kSeg, g.BH()), kRouteThreads, psmem, stream>>>(sel, g.nb, keep_k, order);
     } else {
       identity_order<<<dim3((g.nb + 255) / 256, g.BH()), 256, 0, stream>>>(g.nb, order);

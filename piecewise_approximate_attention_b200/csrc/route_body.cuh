@@ -204,8 +204,7 @@ constexpr size_t route_smem_floats(int nb) {
 // of kSeg consecutive blocks, one CTA each; inside a segment a greedy pass in index order pairs each
 // unpaired block i with the unpaired block p of the same segment (p > i) whose selection shares the
 // most key blocks with S_i (ties to the nearer p).  Pairs fill the segment's range of the order
-// first, in order of decreasing union size, blocks left without a partner follow, so no tile
-// straddles two segments (a full segment
+// first, blocks left without a partner follow, so no tile straddles two segments (a full segment
 // holds an even count).  The attention result does not depend on the order; only the union of S_i
 // and S_p, which one tile iterates over, does.  Bitmaps of the selections live in shared memory.
 constexpr int kSeg = 128;
@@ -228,7 +227,6 @@ __device__ __forceinline__ void pair_segment(const int32_t* __restrict__ sel, in
   uint32_t* bits = psm;                                                  // [nwords][kSeg]
   uint16_t* ov = reinterpret_cast<uint16_t*>(bits + kSeg * nwords);     // [kSeg][kSeg], a < b used
   int32_t* singles = reinterpret_cast<int32_t*>(ov + kSeg * kSeg);      // [kSeg]
-  uint32_t* pairs = reinterpret_cast<uint32_t*>(singles + kSeg);        // [kSeg / 2]: a | b << 8 | overlap << 16
   __shared__ int npos_s, nsingle_s;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s0 = seg * kSeg, n = min(kSeg, nb - s0);
@@ -294,7 +292,10 @@ __device__ __forceinline__ void pair_segment(const int32_t* __restrict__ sel, in
         u3 |= w == 3 ? bit : 0u;
       }
       if (key) {
-        if (lane == 0) pairs[npos >> 1] = (uint32_t)a | ((uint32_t)pb << 8) | (((key >> 8) - 1u) << 16);
+        if (lane == 0) {
+          out[npos] = s0 + a;
+          out[npos + 1] = s0 + pb;
+        }
         npos += 2;
       } else {
         if (lane == 0) singles[nsingle] = s0 + a;
@@ -307,25 +308,11 @@ __device__ __forceinline__ void pair_segment(const int32_t* __restrict__ sel, in
     }
   }
   __syncthreads();
-  // pairs in order of decreasing union |S_a| + |S_b| - overlap, i.e. increasing overlap (ties in
-  // pairing order): the attention kernel, launched in this order for short sequences, starts its
-  // longest tiles first, which shortens the tail of its last wave
-  const int npairs = npos_s >> 1;
-  for (int e = threadIdx.x; e < npairs; e += kRouteThreads) {
-    const uint32_t me = pairs[e], mo = me >> 16;
-    int rank = 0;
-    for (int u = 0; u < npairs; ++u) {
-      const uint32_t uo = pairs[u] >> 16;
-      rank += (uo < mo || (uo == mo && u < e)) ? 1 : 0;
-    }
-    out[2 * rank] = s0 + (int)(me & 255u);
-    out[2 * rank + 1] = s0 + (int)((me >> 8) & 255u);
-  }
   for (int e = threadIdx.x; e < nsingle_s; e += kRouteThreads) out[npos_s + e] = singles[e];
 }
 
 __host__ __device__ constexpr size_t pair_smem_bytes(int nb) {
-  return (size_t)kSeg * ((nb + 31) / 32) * 4 + (size_t)kSeg * kSeg * 2 + (size_t)kSeg * 4 + (size_t)kSeg / 2 * 4;
+  return (size_t)kSeg * ((nb + 31) / 32) * 4 + (size_t)kSeg * kSeg * 2 + (size_t)kSeg * 4;
 }
 
 }  // namespace

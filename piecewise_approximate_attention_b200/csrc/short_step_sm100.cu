@@ -208,7 +208,7 @@ template <bool kDiff>
 cudaError_t launch_short(const KVMaps& maps, const ShortParams& sp, int nparts, int bh, cudaStream_t stream,
                          bool* launched) {
   const size_t smem = short_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(short_step_sm100<kDiff>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(short_step_sm100<kDiff>), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nparts, bh, 1);

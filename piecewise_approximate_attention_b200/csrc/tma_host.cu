@@ -1,8 +1,11 @@
-// Host-side TMA descriptor encoding (cuTensorMapEncodeTiled through the runtime's driver entry
-// point, so the library needs no link-time dependency on libcuda).
+// Host-side helpers: TMA descriptor encoding (cuTensorMapEncodeTiled through the runtime's driver
+// entry point, so the library needs no link-time dependency on libcuda) and the kernels'
+// dynamic-shared-memory attribute, set once per kernel and device.
 #include <cudaTypedefs.h>
 
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 
@@ -22,7 +25,49 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+std::mutex g_attr_mu;
+// (kernel, CUDA context id) -> bytes already allowed; keyed by context so that a context created
+// after cudaDeviceReset sets the attribute again
+std::map<std::pair<const void*, unsigned long long>, size_t> g_attr_set;
+
 }  // namespace
+
+// Unique id of the calling thread's current CUDA context (0 if none is current or the driver
+// cannot say).  Driver entry points through the runtime: no link-time dependency on libcuda.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+cudaError_t set_max_dynamic_smem(const void* fn, size_t bytes) {
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  if (ctx != 0) {
+    auto it = g_attr_set.find({fn, ctx});
+    if (it != g_attr_set.end() && it->second >= bytes) return cudaSuccess;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (ctx != 0) g_attr_set[{fn, ctx}] = bytes;
+  return cudaSuccess;
+}
 
 bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
                     uint32_t box_rows) {

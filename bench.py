@@ -249,21 +249,13 @@ def run_ours(args, rank, world, local_rank):
         o = torch.empty_like(qd)
     torch.cuda.synchronize()
 
-    fused = p.fused_short_step()
-
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        if fused:
-            # short sequences: pre-computation and routing in one cluster launch (timed as pre-compute)
-            p.precompute_route(qd, kd, vd, stream=stream)
-            if evs:
-                evs[1].record(stream)
-        else:
-            p.precompute(qd, kd, vd, stream)
-            if evs:
-                evs[1].record(stream)
-            p.route(stream=stream)
+        p.precompute(qd, kd, vd, stream)
+        if evs:
+            evs[1].record(stream)
+        p.route(stream=stream)
         if evs:
             evs[2].record(stream)
         p.attention(qd, kd, vd, o, stream=stream)
@@ -581,10 +573,9 @@ SHORT_WORKLOADS = ("image-dit", "sweep-L8192-s0.875")
 
 def short_sequences(dev, reps: int = 30):
     """Short sequences, where per-launch overhead and the pre-computation weigh most: the full
-    step (pre-compute and route in one cluster launch + attention) launched call by call and
-    replayed as one CUDA graph, its parts (the fused pre-compute + route, and the separate
-    pre-compute and route calls), and the library's dense attention on the same inputs, timed
-    interleaved (medians).  Outside the timed region."""
+    step launched call by call and replayed as one CUDA graph (with the separate pre-compute and
+    route kernels, and with them fused into one cluster launch), its parts, and the library's
+    dense attention on the same inputs, timed interleaved (medians).  Outside the timed region."""
     import torch
     from piecewise_approximate_attention_b200.runtime import Pisa
     from piecewise_approximate_attention_b200.workloads import WORKLOADS, make_qkv
@@ -597,13 +588,13 @@ def short_sequences(dev, reps: int = 30):
         p = Pisa(B, H, L, d, w.block, w.keep_k, w.lam, w.dtype, 1.0, dev)
         o = torch.empty_like(q)
         graph = p.capture(q, k, v, o)
-        graph_sep = p.capture(q, k, v, o, fused=False)
+        graph_fused = p.capture(q, k, v, o, fused=True)
         dense = Pisa(B, H, L, d, w.block, p.nb, w.lam, w.dtype, 1.0, dev, pair=False)
         dense.precompute(q, k, v)
         dense.route()
         arms = {"step_launches": lambda: p(q, k, v, o), "step_graph": graph.replay,
-                "step_graph_separate_precompute_route": graph_sep.replay,
-                "precompute_route_fused": lambda: p.precompute_route(q, k, v),
+                "step_graph_fused_precompute_route": graph_fused.replay,
+                "precompute_route_fused": lambda: p.precompute_route(q, k, v, fused=True),
                 "precompute": lambda: p.precompute(q, k, v), "route": lambda: p.route(),
                 "attention": lambda: p.attention(q, k, v, o), "dense_attention": lambda: dense.attention(q, k, v, o)}
         with NvmlClock(dev.index or 0) as nclk:
@@ -614,7 +605,7 @@ def short_sequences(dev, reps: int = 30):
                      "p10_p90_ms_step_graph": [st["step_graph"]["p10_ms"], st["step_graph"]["p90_ms"]],
                      "sm_mhz": st["step_graph"]["sm_mhz"],
                      "speedup_step_vs_dense": round(st["dense_attention"]["median_ms"] / st["step_graph"]["median_ms"], 3)}
-        del graph, graph_sep, p, dense
+        del graph, graph_fused, p, dense
     return out
 
 
@@ -759,7 +750,7 @@ def profile_case(a):
     for _ in range(a.iters):
         if perm is None:
             if a.fused:
-                p.precompute_route(q, k, v)
+                p.precompute_route(q, k, v, fused=True)
             else:
                 p.precompute(q, k, v)
                 p.route()

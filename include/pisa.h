@@ -195,18 +195,21 @@ PISA_API pisa_status pisa_precompute_noalloc(const pisa_shape* shape, const void
 PISA_API pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t keep_k, float lambda,
                        int32_t* sel, int32_t* order, float* scores, pisa_stream_t stream);
 
-/* pisa_precompute followed by pisa_route, with the same arguments, results and errors, in as few
- * launches as the shape allows (§1 문제 정의 and §4 실험 결과: the method must keep its edge at short
- * sequences, where the fixed cost of pre-computation and routing weighs most).  For bf16 inputs
- * (PISA_BF16, PISA_BF16_FP8QK) with nb <= 128 it is one launch of a thread-block cluster per
- * (batch, head), whose CTAs meet at hardware cluster barriers between the passes (the e4m3 copies
- * add their quantization launch); every array it writes
- * is bit-identical to what the two separate calls write.  Otherwise, or when the device cannot
- * schedule that cluster, it makes the separate calls.  ws as for pisa_precompute. */
+/* pisa_precompute followed by pisa_route, with the same arguments, results and errors.
+ * flags = 0: the separate calls.  flags = PISA_PRECOMPUTE_ROUTE_FUSED: for bf16 inputs (PISA_BF16,
+ * PISA_BF16_FP8QK) with nb <= 128 (short sequences, where the fixed cost of pre-computation and
+ * routing weighs most: §1 문제 정의, §4 실험 결과), one launch of a thread-block cluster per (batch,
+ * head) whose CTAs meet at hardware cluster barriers between the passes (the e4m3 copies add their
+ * quantization launch); every array it writes is bit-identical to what the separate calls write.
+ * Otherwise, or when the device cannot make every head's cluster co-resident, it makes the
+ * separate calls.  Measured on B200 the fused launch is not faster than the separate kernels
+ * replayed as a CUDA graph (each pass is bound by its own per-CTA latency, not by launch gaps), so
+ * it is not the default.  Any other flags value: PISA_ERR_INVALID_ARG.  ws as for pisa_precompute. */
+#define PISA_PRECOMPUTE_ROUTE_FUSED 1
 PISA_API pisa_status pisa_precompute_route(const pisa_shape* shape, const void* q, const void* k, const void* v,
                                            const pisa_stats* stats, int32_t keep_k, float lambda, int32_t* sel,
                                            int32_t* order, float* scores, void* ws, size_t ws_bytes,
-                                           pisa_stream_t stream);
+                                           int32_t flags, pisa_stream_t stream);
 
 /* Exact-or-approximate attention (§2: o_t = N_t / D_t and the numerator equation; 하드웨어 구현
  * stages 1-3: exact selected blocks, zeroth-order scan of the other blocks, global first-order

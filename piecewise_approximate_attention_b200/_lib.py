@@ -66,7 +66,7 @@ def lib() -> ctypes.CDLL:
             "pisa_precompute_zeroth_order": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, sz, vp]),
             "pisa_route": (i32, [P(PisaShape), P(PisaStats), i32, f32, vp, vp, vp, vp]),
             "pisa_precompute_route": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), i32, f32, vp, vp, vp, vp, sz,
-                                            vp]),
+                                            i32, vp]),
             "pisa_attention": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp, vp, i32, i32, vp, vp, sz, vp]),
             "pisa_read_device_error": (i32, [vp, P(i32), vp]),
             "pisa_status_string": (ctypes.c_char_p, [i32]),
@@ -223,12 +223,16 @@ def pisa_route(shape: PisaShape, stats: Stats, keep_k: int, lam: float, sel, ord
                             _ptr(order), _ptr(scores), _stream(stream)), "pisa_route")
 
 
+PISA_PRECOMPUTE_ROUTE_FUSED = 1
+
+
 def pisa_precompute_route(shape: PisaShape, q, k, v, stats: Stats, keep_k: int, lam: float, sel, order, scores, ws,
-                          stream=None):
-    """pisa_precompute then pisa_route; one cluster launch for bf16 inputs with nb <= 128."""
+                          fused: bool = False, stream=None):
+    """pisa_precompute then pisa_route; with fused, one cluster launch for bf16 inputs with nb <= 128."""
     _check(lib().pisa_precompute_route(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(stats.c),
                                        int(keep_k), float(lam), _ptr(sel), _ptr(order), _ptr(scores), _ptr(ws),
-                                       ws.numel(), _stream(stream)), "pisa_precompute_route")
+                                       ws.numel(), PISA_PRECOMPUTE_ROUTE_FUSED if fused else 0, _stream(stream)),
+           "pisa_precompute_route")
 
 
 def pisa_attention(shape: PisaShape, q, k, v, stats: Stats, sel, order, keep_k: int, mode: int, o, ws, stream=None):

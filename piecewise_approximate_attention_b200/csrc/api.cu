@@ -227,15 +227,19 @@ pisa_status pisa_route(const pisa_shape* shape, const pisa_stats* stats, int32_t
 
 pisa_status pisa_precompute_route(const pisa_shape* shape, const void* q, const void* k, const void* v,
                                   const pisa_stats* stats, int32_t keep_k, float lambda, int32_t* sel,
-                                  int32_t* order, float* scores, void* ws, size_t ws_bytes, pisa_stream_t stream) {
+                                  int32_t* order, float* scores, void* ws, size_t ws_bytes, int32_t flags,
+                                  pisa_stream_t stream) {
   Dims g;
   pisa_status s = validate_precompute(shape, q, k, v, stats, &g);
   if (s != PISA_OK) return s;
   if (!ws || !aligned16(ws) || ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   if ((s = check_route_args(g, keep_k, lambda, sel, order, scores)) != PISA_OK) return s;
+  if (flags != 0 && flags != PISA_PRECOMPUTE_ROUTE_FUSED) return PISA_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   bool launched = false;
-  cudaError_t e = launch_short_step_sm100(g, q, k, v, *stats, ws, keep_k, lambda, sel, order, scores, cs, &launched);
+  cudaError_t e = cudaSuccess;
+  if (flags == PISA_PRECOMPUTE_ROUTE_FUSED)
+    e = launch_short_step_sm100(g, q, k, v, *stats, ws, keep_k, lambda, sel, order, scores, cs, &launched);
   if (e != cudaSuccess) return PISA_ERR_CUDA;
   if (launched) {
     if (g.dtype == PISA_BF16_FP8QK) e = launch_quantize_fp8(g, q, k, *stats, cs);

@@ -48,17 +48,19 @@ class Pisa:
             C.pisa_precompute_zeroth_order(self.shape, q, k, v, self.stats, self.ws, stream)
 
     def fused_short_step(self) -> bool:
-        """Whether precompute_route runs as one cluster launch (bf16 inputs, head_dim 128, nb <= 128)."""
+        """Whether precompute_route(fused=True) is one cluster launch (bf16 inputs, head_dim 128,
+        nb <= 128; the device must also fit every head's cluster at once)."""
         return self.first_order and self.tdtype != self._torch_f32 and self.shape.head_dim == 128 and self.nb <= 128
 
-    def precompute_route(self, q, k, v, scores=None, stream=None):
-        """Pre-computation and routing; for short sequences one cluster launch (same results)."""
+    def precompute_route(self, q, k, v, scores=None, stream=None, fused: bool = False):
+        """Pre-computation and routing through pisa_precompute_route: the separate kernels, or with
+        ``fused`` (short sequences) one cluster launch; the results are the same either way."""
         if not self.first_order:
             self.precompute(q, k, v, stream)
             self.route(scores, stream)
             return
         C.pisa_precompute_route(self.shape, q, k, v, self.stats, self.keep_k, self.lam, self.sel, self.order, scores,
-                                self.ws, stream)
+                                self.ws, fused, stream)
 
     def route(self, scores=None, stream=None):
         C.pisa_route(self.shape, self.stats, self.keep_k, self.lam, self.sel, self.order, scores, stream)
@@ -77,12 +79,13 @@ class Pisa:
         self.attention(q, k, v, o, stream=stream)
         return o
 
-    def capture(self, q, k, v, o, fused: bool = True):
+    def capture(self, q, k, v, o, fused: bool = False):
         """Records one full step (pre-computation, routing, attention of q, k, v into o) as a CUDA
         graph and returns it; ``graph.replay()`` then re-runs the step on whatever the same
         buffers hold, with one launch from the host.  The buffers must stay allocated while the
-        graph is used.  The step runs once eagerly first (outside the capture).  ``fused=False``
-        records the separate pre-computation and routing calls instead of precompute_route."""
+        graph is used.  The step runs once eagerly first (outside the capture).  ``fused=True``
+        records the fused pre-computation and routing (short sequences) instead of the separate
+        calls."""
         import torch
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
@@ -91,25 +94,18 @@ class Pisa:
         torch.cuda.current_stream(self.device).wait_stream(side)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side):
-            if fused:
-                self.precompute_route(q, k, v)
-            else:
-                self.precompute(q, k, v)
-                self.route()
+            self.precompute_route(q, k, v, fused=fused)
             self.attention(q, k, v, o)
         return graph
 
     def launches_per_step(self) -> int:
         """Kernels one __call__ enqueues: pre-compute 3 (2 zeroth-order only on the bf16 path, 1 on
-        the fp32 path; +3 e4m3 quantizations), routing 1 (+1 pairing) -- or, for short bf16
-        sequences, pre-compute and routing in 1 cluster launch -- and attention 1 (+1 for the
+        the fp32 path; +3 e4m3 quantizations), routing 1 (+1 pairing), attention 1 (+1 for the
         per-block first-order kernel on the bf16 path)."""
         extra = 1 if (self.mode == C.PISA_MODE_PER_BLOCK and self.tdtype != self._torch_f32 and
                       self.keep_k < self.nb) else 0
         pre = 3 if self.first_order else (1 if self.tdtype == self._torch_f32 else 2)
         route = 1 + (1 if self.order is not None else 0)
-        if self.fused_short_step():
-            pre, route = 1, 0          # pre-computation and routing in one cluster launch
         return pre + (3 if self.fp8 else 0) + route + 1 + extra
 
     def device_error(self, stream=None):

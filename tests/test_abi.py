@@ -235,3 +235,17 @@ def test_headers_are_plain_c_and_the_library_links_from_c(tmp_path):
     res = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0, res.stderr
     assert "c consumer ok: abi 6" in res.stdout
+
+
+def test_precompute_route_checks_its_flags():
+    L = C.lib()
+    sh = _shape()
+    st = _fake_stats(sh)
+    ws = C.pisa_workspace_bytes(sh)
+    P = 1 << 28
+    for flags in (2, -1, 3):
+        assert L.pisa_precompute_route(ctypes.byref(sh), P, P, P, ctypes.byref(st), 4, 0.5, P, None, None, P, ws, flags,
+                                       None) == C.PISA_ERR_INVALID_ARG
+    # the route arguments are checked as by pisa_route, before anything is enqueued
+    assert L.pisa_precompute_route(ctypes.byref(sh), P, P, P, ctypes.byref(st), 17, 0.5, P, None, None, P, ws, 0,
+                                   None) == C.PISA_ERR_INVALID_ARG

@@ -1,7 +1,8 @@
 """Pre-computation and routing in one launch for short sequences (needs a B200).
 
-pisa_precompute_route runs, for bf16 inputs with at most 128 key blocks, one thread-block cluster per
-head that does both passes of the pre-computation, the Hbar reduction, the routing and the pairing.
+pisa_precompute_route with PISA_PRECOMPUTE_ROUTE_FUSED runs, for bf16 inputs with at most 128 key
+blocks, one thread-block cluster per head that does both passes of the pre-computation, the Hbar
+reduction, the routing and the pairing.
 It uses the same code and summation orders as the separate calls, so every array it writes must be
 bit-identical to pisa_precompute followed by pisa_route; longer sequences fall back to those calls.
 """
@@ -50,7 +51,7 @@ def test_fused_equals_separate_calls(name, w, keep_k, lam, dtype, with_H):
     sb = torch.full_like(sa, float("nan"))
     a.precompute(q, k, v)
     a.route(scores=sa)
-    b.precompute_route(q, k, v, scores=sb)
+    b.precompute_route(q, k, v, scores=sb, fused=True)
     torch.cuda.synchronize()
     assert a.device_error() == (C.PISA_OK, 0) and b.device_error() == (C.PISA_OK, 0)
     for f in STATS:
@@ -78,7 +79,7 @@ def test_fused_step_graph_replay():
     ref.route()
     ref.attention(q, k, v, o_ref)
     o = torch.empty_like(q)
-    g = p.capture(q, k, v, o)
+    g = p.capture(q, k, v, o, fused=True)
     for _ in range(2):
         o.fill_(float("nan"))
         g.replay()

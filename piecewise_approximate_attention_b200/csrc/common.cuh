@@ -92,6 +92,8 @@ cudaError_t set_max_dynamic_smem(const void* fn, size_t bytes);
 // Unique id of the calling thread's current CUDA context, 0 if none is current (or the driver
 // cannot say).  Host caches of per-context state key on it.
 unsigned long long current_context_id();
+// Number of SMs of the current device (cached per device ordinal).
+cudaError_t sm_count(int* n);
 
 // Argument checks of pisa_precompute other than its workspace (shape, q, k, v, stats); fills *g.
 // Enqueues nothing.  Shared by the entry points that run the pre-computation.
@@ -104,8 +106,10 @@ cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, 
                                    const pisa_stats& st, void* ws, bool first_order, cudaStream_t stream);
 cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v,
                                     const pisa_stats& st, void* ws, bool first_order, cudaStream_t stream);
+// pdl: launch with programmatic stream serialization (the kernel waits for the previous kernel of
+// the stream before it reads anything, and lets the next one start at once).
 cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const float* vmax,
-                               const pisa_stats& st, cudaStream_t stream);
+                               const pisa_stats& st, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream);
 // Pre-computation + routing in one cluster launch (bf16 inputs, d = 128, nb <= 128).  *launched is

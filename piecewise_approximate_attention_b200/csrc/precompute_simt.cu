@@ -104,12 +104,19 @@ __global__ void __launch_bounds__(kThreads) stats_partial(const T* __restrict__ 
 // Per head: Hbar = (sum of the group partials of H_j, in order) / nb, its bf16 operand copy, and
 // (when vmax is given) the value scale: the smallest power of two >= max|v| / 256, so that
 // v / vscale and every block sum of it (at most 128 terms) fit comfortably in fp16.
+// One thread per four consecutive elements; the partials are read eight at a time (all loads in
+// flight together) and added in group order, so the sum is the same as a plain loop's.
+// Launched with programmatic stream serialization after the pass that writes the partials, it
+// lets the next kernel start at once and waits for the partials before it reads them.
 template <int D>
 __global__ void __launch_bounds__(kThreads) hbar_reduce(const float* __restrict__ partials, int nparts, int nb,
                                                         float scale, float* __restrict__ hbar,
                                                         __nv_bfloat16* __restrict__ hbar_op,
                                                         const float* __restrict__ vmax, float* __restrict__ vscale) {
-  const int e = blockIdx.x * kThreads + threadIdx.x, bh = blockIdx.y;
+  constexpr int kVec = D * D / 4;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int e4 = blockIdx.x * kThreads + threadIdx.x, bh = blockIdx.y;
   if (vmax && vscale && blockIdx.x == 0 && threadIdx.x == 0) {
     float mx = 0.f;
     for (int i = 0; i < nparts; ++i) mx = fmaxf(mx, vmax[(size_t)bh * nparts + i]);
@@ -117,15 +124,34 @@ __global__ void __launch_bounds__(kThreads) hbar_reduce(const float* __restrict_
     while (mx > 256.f * sc && sc < 0x1p100f) sc *= 2.f;
     vscale[bh] = sc;
   }
-  if (e >= D * D) return;
-  const float* p = partials + (size_t)bh * nparts * D * D + e;
-  float s = 0.f;
-  for (int i = 0; i < nparts; ++i) s += p[(size_t)i * D * D];
-  const float h = s / (float)nb;
-  hbar[(size_t)bh * D * D + e] = h;
+  if (e4 >= kVec) return;
+  const float4* p = reinterpret_cast<const float4*>(partials + (size_t)bh * nparts * D * D) + e4;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < nparts; i += 8) {
+    float4 x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (i + u < nparts) x[u] = __ldcg(p + (size_t)(i + u) * kVec);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (i + u < nparts) {
+        s.x += x[u].x;
+        s.y += x[u].y;
+        s.z += x[u].z;
+        s.w += x[u].w;
+      }
+    }
+  }
+  const float fnb = (float)nb;
+  const float4 h = make_float4(s.x / fnb, s.y / fnb, s.z / fnb, s.w / fnb);
+  reinterpret_cast<float4*>(hbar + (size_t)bh * D * D)[e4] = h;
   if (hbar_op) {
-    const int a = e / D, c = e % D;
-    hbar_op[(size_t)bh * D * D + c * D + a] = __float2bfloat16_rn(scale * h);
+    const int a = (4 * e4) / D, c = (4 * e4) % D;
+    __nv_bfloat16* op = hbar_op + (size_t)bh * D * D + a;
+    op[(size_t)(c + 0) * D] = __float2bfloat16_rn(scale * h.x);
+    op[(size_t)(c + 1) * D] = __float2bfloat16_rn(scale * h.y);
+    op[(size_t)(c + 2) * D] = __float2bfloat16_rn(scale * h.z);
+    op[(size_t)(c + 3) * D] = __float2bfloat16_rn(scale * h.w);
   }
 }
 
@@ -188,7 +214,7 @@ cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, cons
   }
   stats_partial<T, D, true><<<dim3(nparts, g.BH()), kThreads, smem_a, stream>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g.L, g.block, g.nb, st, partials);
-  hbar_reduce<D><<<dim3((D * D + kThreads - 1) / kThreads, g.BH()), kThreads, 0, stream>>>(
+  hbar_reduce<D><<<dim3((D * D / 4 + kThreads - 1) / kThreads, g.BH()), kThreads, 0, stream>>>(
       partials, nparts, g.nb, g.scale, st.hbar, static_cast<__nv_bfloat16*>(st.hbar_op), nullptr, nullptr);
   cov_norm<T, D><<<dim3(g.nb, g.BH()), kThreads, smem_c, stream>>>(
       static_cast<const T*>(k), static_cast<const T*>(v), g.L, g.block, g.nb, st);
@@ -198,15 +224,21 @@ cudaError_t run(const Dims& g, const void* q, const void* k, const void* v, cons
 }  // namespace
 
 cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const float* vmax,
-                               const pisa_stats& st, cudaStream_t stream) {
-  dim3 grid((g.d * g.d + kThreads - 1) / kThreads, g.BH());
+                               const pisa_stats& st, cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((g.d * g.d / 4 + kThreads - 1) / kThreads, g.BH());
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  __nv_bfloat16* hop = static_cast<__nv_bfloat16*>(st.hbar_op);
   if (g.d == 64)
-    hbar_reduce<64><<<grid, kThreads, 0, stream>>>(partials, nparts, g.nb, g.scale, st.hbar,
-                                                   static_cast<__nv_bfloat16*>(st.hbar_op), vmax, st.vscale);
-  else
-    hbar_reduce<128><<<grid, kThreads, 0, stream>>>(partials, nparts, g.nb, g.scale, st.hbar,
-                                                    static_cast<__nv_bfloat16*>(st.hbar_op), vmax, st.vscale);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, hbar_reduce<64>, partials, nparts, g.nb, g.scale, st.hbar, hop, vmax, st.vscale);
+  return cudaLaunchKernelEx(&cfg, hbar_reduce<128>, partials, nparts, g.nb, g.scale, st.hbar, hop, vmax, st.vscale);
 }
 
 cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,

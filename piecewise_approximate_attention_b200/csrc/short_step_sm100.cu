@@ -94,15 +94,18 @@ __global__ void __launch_bounds__(kShortThreads, 1) short_step_sm100(const __gri
   const uint32_t tmem = tmem_base;
 
   // ---- 1. pass A of this CTA's group ----
-  stats_a_body<true>(maps, p, sm.a, tmem, rank, bh, nparts, p.partials + ((size_t)bh * nparts + rank) * D * D);
+  const int unit = bh * nparts + rank;                // group `rank` of head bh
+  stats_a_body<true>(maps, p, sm.a, tmem, unit, unit + 1, nparts);
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_inval(&sm.a.full[s]);
       mbar_inval(&sm.a.empty[s]);
       mbar_inval(&sm.a.sums_full[s]);
       mbar_inval(&sm.a.sums_empty[s]);
+      mbar_inval(&sm.a.acc_full[s]);
+      mbar_inval(&sm.a.acc_empty[s]);
     }
-    mbar_inval(&sm.a.acc_done);
+    mbar_inval(&sm.a.drain);
   }
   cluster_sync_all();
 
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(kShortThreads, 1) short_step_sm100(const __gri
   cluster_sync_all();      // Hbar and the value scale written
 
   // ---- 3. pass B of this CTA's group ----
-  cov_norm_body<kDiff>(maps, p, sm.b, tmem, rank, bh);
+  cov_norm_body<kDiff>(maps, p, sm.b, tmem, unit, unit + 1, nparts);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesB; ++s) {
       mbar_inval(&sm.b.full[s]);

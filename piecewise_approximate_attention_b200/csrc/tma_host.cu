@@ -1,8 +1,9 @@
 // Host-side helpers: TMA descriptor encoding (cuTensorMapEncodeTiled through the runtime's driver
-// entry point, so the library needs no link-time dependency on libcuda) and the kernels'
-// dynamic-shared-memory attribute, set once per kernel and device.
+// entry point, so the library needs no link-time dependency on libcuda), the kernels'
+// dynamic-shared-memory attribute, set once per kernel and device, and the device's SM count.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -54,6 +55,18 @@ unsigned long long current_context_id() {
   unsigned long long id = 0;
   if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
   return id;
+}
+
+cudaError_t sm_count(int* n) {
+  static std::atomic<int> cache[64];     // per device ordinal; 0 = not asked yet
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < 64;
+  if (cached && (*n = cache[dev].load(std::memory_order_relaxed)) > 0) return cudaSuccess;
+  if ((e = cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if (cached) cache[dev].store(*n, std::memory_order_relaxed);
+  return cudaSuccess;
 }
 
 cudaError_t set_max_dynamic_smem(const void* fn, size_t bytes) {

@@ -16,14 +16,14 @@
 namespace pisa {
 namespace {
 
-template <int D, int kRows>
+template <int D, int kRows, int kCols>
 __global__ void __launch_bounds__(kRouteThreads, 2) route_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
                                                               const float* __restrict__ M, int L, int block, int nb,
                                                               float scale, int keep_k, float lam,
                                                               int32_t* __restrict__ sel, float* __restrict__ scores) {
   extern __shared__ __align__(16) float smem[];
   const int i0 = blockIdx.x * kRows;
-  route_rows<D, kRows>(qbar, kbar, M, L, block, nb, scale, keep_k, lam, sel, scores, blockIdx.y, i0,
+  route_rows<D, kRows, kCols>(qbar, kbar, M, L, block, nb, scale, keep_k, lam, sel, scores, blockIdx.y, i0,
                        min(kRows, nb - i0), smem);
 }
 
@@ -39,15 +39,15 @@ __global__ void identity_order(int nb, int32_t* __restrict__ order) {
     order[(size_t)bh * nb + i] = i;
 }
 
-template <int D, int kRows>
+template <int D, int kRows, int kCols>
 cudaError_t launch_route_kernel(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                                 float* scores, cudaStream_t stream) {
-  const size_t smem = route_smem_floats<D, kRows>(g.nb) * sizeof(float);
+  const size_t smem = route_smem_floats<D, kRows, kCols>(g.nb) * sizeof(float);
   cudaError_t e;
-  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(route_kernel<D, kRows>), smem)))
+  if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(route_kernel<D, kRows, kCols>), smem)))
     return e;
   // lambda == 0 drops the M term: M is not read (it may be unwritten)
-  route_kernel<D, kRows><<<dim3((g.nb + kRows - 1) / kRows, g.BH()), kRouteThreads, smem, stream>>>(
+  route_kernel<D, kRows, kCols><<<dim3((g.nb + kRows - 1) / kRows, g.BH()), kRouteThreads, smem, stream>>>(
       st.qbar, st.kbar, lam > 0.f ? st.M : nullptr, g.L, g.block, g.nb, g.scale, keep_k, lam, sel, scores);
   return cudaGetLastError();
 }
@@ -57,13 +57,16 @@ cudaError_t launch_route_kernel(const Dims& g, const pisa_stats& st, int keep_k,
 cudaError_t launch_route(const Dims& g, const pisa_stats& st, int keep_k, float lam, int32_t* sel,
                          int32_t* order, float* scores, cudaStream_t stream) {
   cudaError_t e;
-  // 16 query blocks per CTA while their score rows fit comfortably in shared memory, else 8
-  if (g.d == 64)
-    e = g.nb <= 2048 ? launch_route_kernel<64, 16>(g, st, keep_k, lam, sel, scores, stream)
-                     : launch_route_kernel<64, 8>(g, st, keep_k, lam, sel, scores, stream);
+  // 16 query blocks per CTA while their score rows fit comfortably in shared memory, else 8; one or
+  // two centroids per thread (route_cols)
+  const bool two = route_cols(g.nb) == 2;
+  if (g.d == 64)   // (head_dim 64: one centroid per thread up to nb = 2048, which fits its registers)
+    e = g.nb > 2048 ? launch_route_kernel<64, 8, 2>(g, st, keep_k, lam, sel, scores, stream)
+                    : launch_route_kernel<64, 16, 1>(g, st, keep_k, lam, sel, scores, stream);
   else
-    e = g.nb <= 2048 ? launch_route_kernel<128, 16>(g, st, keep_k, lam, sel, scores, stream)
-                     : launch_route_kernel<128, 8>(g, st, keep_k, lam, sel, scores, stream);
+    e = g.nb > 2048 ? launch_route_kernel<128, 8, 2>(g, st, keep_k, lam, sel, scores, stream)
+        : two       ? launch_route_kernel<128, 16, 2>(g, st, keep_k, lam, sel, scores, stream)
+                    : launch_route_kernel<128, 16, 1>(g, st, keep_k, lam, sel, scores, stream);
   if (e != cudaSuccess) return e;
   if (order) {
     if (g.block == 64 && keep_k > 0 && g.nb > 2) {

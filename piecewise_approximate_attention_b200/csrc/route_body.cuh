@@ -80,27 +80,42 @@ __device__ void warp_topk(const uint32_t* u, int nb, int keep_k, uint32_t* hist,
   }
 }
 
-// Scores of kRows query blocks against all nb centroids: k̄ is streamed through shared memory in
-// tiles of kTileJ = 4 * kRouteThreads / kRows rows (coalesced float4 loads, rows padded by 4 floats so
-// the float4 reads of 32 different rows are conflict-free); each thread accumulates 4 query blocks
-// x 1 centroid.
+// Scores of kRows query blocks against all nb centroids.  Each thread accumulates 8 query blocks x
+// kCols centroids (jj, and jj + kRouteThreads / (kRows / 8) when kCols = 2); k̄ is streamed through
+// shared memory in tiles of route_tile_j centroids x route_chunk columns (coalesced float4 loads,
+// rows padded by 4 floats so that the float4 reads of 8 consecutive rows cover all 32 banks), the
+// next chunk being loaded into registers while the current one is used.  Two centroids per thread
+// halve the shared-memory reads per FMA but double the tile, which short rows of centroids (nb up
+// to 256) would mostly leave empty.  Every score is summed over the columns in order, four at a
+// time as fmaf(q.x, k.x, fmaf(q.y, k.y, fmaf(q.z, k.z, fmaf(q.w, k.w, acc)))).
 template <int kRows>
-constexpr int tile_j() { return 4 * kRouteThreads / kRows; }
+constexpr int route_group_threads() { return kRouteThreads / (kRows / 8); }
+template <int kRows, int kCols>
+constexpr int route_tile_j() { return kCols * route_group_threads<kRows>(); }
+template <int kRows>
+constexpr int route_chunk() { return kRows == 16 ? 32 : 16; }
+// centroids per thread for a head of nb key blocks
+inline int route_cols(int nb) { return nb > 256 ? 2 : 1; }
 
 // Body: routes query blocks [i0, i0 + rows) (rows <= kRows) of head bh with kRouteThreads threads;
 // `smem` holds route_smem_floats<D, kRows>(nb) floats (16-byte aligned).  qbar, kbar and M are not
 // __restrict__: the fused short-sequence kernel writes them earlier in the same launch, so they
 // must be read through the coherent path.
-template <int D, int kRows>
+template <int D, int kRows, int kCols>
 __device__ __forceinline__ void route_rows(const float* qbar, const float* kbar, const float* M, int L, int block,
                                            int nb, float scale,
                                            int keep_k, float lam, int32_t* __restrict__ sel, float* __restrict__ scores,
                                            int bh, int i0, int rows, float* smem) {
-  constexpr int kTileJ = tile_j<kRows>();
+  static_assert(kRows == 8 || kRows == 16, "8 query blocks per thread, one or two groups");
+  static_assert(kCols == 1 || kCols == 2, "one or two centroids per thread");
+  constexpr int kTPG = route_group_threads<kRows>();       // threads per group of 8 query blocks
+  constexpr int kTileJ = route_tile_j<kRows, kCols>();
+  constexpr int kChunk = route_chunk<kRows>();
+  constexpr int kPitch = kChunk + 4;
   float* qs = smem;                                        // [kRows][D]
-  float* ks = qs + kRows * D;                              // [kTileJ][D + 4]
-  float* r = ks + kTileJ * (D + 4);                        // [kRows][nb]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(r + kRows * nb);   // [kRouteWarps][256]
+  float* ks = qs + kRows * D;                              // [kTileJ][kPitch]
+  float* r = ks + kTileJ * kPitch;                         // [kRows][nb]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(r + kRows * nb);   // [kRouteWarps][256]: top-k histograms
   float* red = reinterpret_cast<float*>(hist + kRouteWarps * 256);     // [kRouteWarps]
   float* Ms = red + kRouteWarps;                                       // [nb]: M_j of this head
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,44 +138,62 @@ __device__ __forceinline__ void route_rows(const float* qbar, const float* kbar,
   msum = warp_sum(msum);
   if (lane == 0) red[warp] = msum;
 
-  const int jj = threadIdx.x % kTileJ, g = threadIdx.x / kTileJ;   // centroid column, query group
+  const int jj = threadIdx.x % kTPG, g = threadIdx.x / kTPG;   // centroids jj (+ kTPG); query blocks 8g..8g+7
   const float4* kb4 = reinterpret_cast<const float4*>(kbar + (size_t)bh * nb * D);
-  // the next k̄ tile is loaded into registers while the current one is used
-  constexpr int kLoads = kTileJ * (D / 4) / kRouteThreads;
-  static_assert(kLoads * kRouteThreads == kTileJ * (D / 4), "tile loads per thread");
+  constexpr int kLoads = kTileJ * (kChunk / 4) / kRouteThreads;
+  static_assert(kLoads * kRouteThreads == kTileJ * (kChunk / 4), "tile loads per thread");
   float4 nxt[kLoads];
-  auto load_tile = [&](int j0) {
+  auto load_chunk = [&](int j0, int c0) {
 #pragma unroll
     for (int x = 0; x < kLoads; ++x) {
-      const int idx = threadIdx.x + x * kRouteThreads, jr = idx / (D / 4), a4 = idx % (D / 4);
-      nxt[x] = j0 + jr < nb ? kb4[(size_t)(j0 + jr) * (D / 4) + a4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int idx = threadIdx.x + x * kRouteThreads, jr = idx / (kChunk / 4), a4 = idx % (kChunk / 4);
+      nxt[x] = j0 + jr < nb ? kb4[(size_t)(j0 + jr) * (D / 4) + c0 / 4 + a4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
-  load_tile(0);
+  load_chunk(0, 0);
   for (int j0 = 0; j0 < nb; j0 += kTileJ) {
     const int nj = min(kTileJ, nb - j0);
-    __syncthreads();
+    // a warp whose centroids all lie past nb only helps with the loads
+    const bool live = (jj - lane) < nj;
+    float acc[8][kCols];
 #pragma unroll
-    for (int x = 0; x < kLoads; ++x) {
-      const int idx = threadIdx.x + x * kRouteThreads, jr = idx / (D / 4), a4 = idx % (D / 4);
-      *reinterpret_cast<float4*>(ks + jr * (D + 4) + 4 * a4) = nxt[x];
-    }
-    __syncthreads();
-    if (j0 + kTileJ < nb) load_tile(j0 + kTileJ);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* kr = ks + jj * (D + 4);
-#pragma unroll 8
-    for (int a = 0; a < D; a += 4) {
-      const float4 kv = *reinterpret_cast<const float4*>(kr + a);
+    for (int x = 0; x < 8; ++x)
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const float4 qv = *reinterpret_cast<const float4*>(qs + (4 * g + x) * D + a);
-        acc[x] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, acc[x]))));
+      for (int c = 0; c < kCols; ++c) acc[x][c] = 0.f;
+    for (int c0 = 0; c0 < D; c0 += kChunk) {
+      __syncthreads();
+#pragma unroll
+      for (int x = 0; x < kLoads; ++x) {
+        const int idx = threadIdx.x + x * kRouteThreads, jr = idx / (kChunk / 4), a4 = idx % (kChunk / 4);
+        *reinterpret_cast<float4*>(ks + jr * kPitch + 4 * a4) = nxt[x];
+      }
+      __syncthreads();
+      if (c0 + kChunk < D) load_chunk(j0, c0 + kChunk);
+      else if (j0 + kTileJ < nb) load_chunk(j0 + kTileJ, 0);
+      if (live) {
+        const float* qg = qs + (8 * g) * D + c0;
+#pragma unroll
+        for (int a = 0; a < kChunk; a += 4) {
+          float4 kv[kCols];
+#pragma unroll
+          for (int c = 0; c < kCols; ++c) kv[c] = *reinterpret_cast<const float4*>(ks + (jj + c * kTPG) * kPitch + a);
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const float4 qv = *reinterpret_cast<const float4*>(qg + x * D + a);
+#pragma unroll
+            for (int c = 0; c < kCols; ++c)
+              acc[x][c] = fmaf(qv.x, kv[c].x, fmaf(qv.y, kv[c].y, fmaf(qv.z, kv[c].z, fmaf(qv.w, kv[c].w, acc[x][c]))));
+          }
+        }
       }
     }
-    if (jj < nj) {
 #pragma unroll
-      for (int x = 0; x < 4; ++x) r[(4 * g + x) * nb + j0 + jj] = acc[x];
+    for (int c = 0; c < kCols; ++c) {
+      const int jc = jj + c * kTPG;
+      if (jc < nj) {
+#pragma unroll
+        for (int x = 0; x < 8; ++x) r[(8 * g + x) * nb + j0 + jc] = acc[x][c];
+      }
     }
   }
   __syncthreads();
@@ -194,10 +227,10 @@ __device__ __forceinline__ void route_rows(const float* qbar, const float* kbar,
 }
 
 
-template <int D, int kRows>
+template <int D, int kRows, int kCols>
 constexpr size_t route_smem_floats(int nb) {
-  return (size_t)kRows * D + (size_t)tile_j<kRows>() * (D + 4) + (size_t)kRows * nb + kRouteWarps * 256 + kRouteWarps +
-         (size_t)nb;
+  return (size_t)kRows * D + (size_t)route_tile_j<kRows, kCols>() * (route_chunk<kRows>() + 4) + (size_t)kRows * nb +
+         kRouteWarps * 256 + kRouteWarps + (size_t)nb;
 }
 
 // Query-block pairing for 128-row tiles when block == 64.  The query blocks are cut into segments

@@ -67,10 +67,10 @@ __device__ __forceinline__ void mbar_inval(uint64_t* bar) {
 union alignas(1024) ShortSmem {
   SmemA a;                                    // phase 1
   SmemB b;                                    // phase 3
-  float route[16 * D + 64 * (D + 4) + 16 * 128 + kRouteWarps * 256 + kRouteWarps + 128];   // phase 4
+  float route[route_smem_floats<D, 16, 1>(128)];                                              // phase 4
   uint32_t pair[pair_smem_bytes(128) / 4];                                                 // phase 5
 };
-static_assert(sizeof(ShortSmem::route) / 4 >= route_smem_floats<D, 16>(128), "routing scratch");
+static_assert(sizeof(ShortSmem::route) / 4 >= route_smem_floats<D, 16, 1>(128), "routing scratch");
 
 template <bool kDiff>
 __global__ void __launch_bounds__(kShortThreads, 1) short_step_sm100(const __grid_constant__ KVMaps maps,
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kShortThreads, 1) short_step_sm100(const __gri
   // ---- 4. routing of query blocks [16 rank, 16 rank + 16) ----
   {
     const int i0 = rank * kBlocksPerPart;
-    route_rows<D, kBlocksPerPart>(p.st.qbar, p.st.kbar, sp.lam > 0.f ? p.st.M : nullptr, p.L, p.block, p.nb, p.scale,
+    route_rows<D, kBlocksPerPart, 1>(p.st.qbar, p.st.kbar, sp.lam > 0.f ? p.st.M : nullptr, p.L, p.block, p.nb, p.scale,
                                   sp.keep_k, sp.lam, sp.sel, sp.scores, bh, i0, min(kBlocksPerPart, p.nb - i0),
                                   sm.route);
   }

@@ -131,6 +131,35 @@ def test_full_size_sampled(name, heads, qblocks):
         assert_output(_np(o[0, h])[keep], ref["o"][0, hi][keep], "bf16", what=f"{name} head {h} full pipeline")
 
 
+BOUNDARY = [
+    # 256 key blocks (one centroid per routing thread) and 257 (two, and a last group of one block);
+    # 10 heads x 16 / 17 groups: more pre-computation groups than SMs, heads split across CTAs
+    ("nb256", (4, 64, 64), 0),
+    ("nb257", (4, 64, 64), 64),
+]
+
+
+@pytest.mark.parametrize("name,grid,text", BOUNDARY, ids=[b[0] for b in BOUNDARY])
+def test_router_blocking_and_persistent_groups(name, grid, text):
+    """Statistics, selections and outputs against the oracle on both sides of the router's switch
+    from one to two centroids per thread, with a persistent pre-computation grid whose groups do
+    not divide evenly over the CTAs."""
+    w = Workload(name, 1, 10, grid, text, 128, 64, 0.875, 0.5, "bf16", seed=3)
+    q, k, v = make_qkv(w)
+    p, o, scores, qkv = _run(w, q, k, v)
+    assert p.nb == (256 if text == 0 else 257)
+    hs = [0, 5, 9]
+    qblocks = [0, 127, p.nb - 1]
+    ref = O.pisa(_np(q[:, hs]), _np(k[:, hs]), _np(v[:, hs]), w.block, w.keep_k, w.lam, qblocks=qblocks)
+    rows = rows_of_blocks(w.seq_len, w.block, qblocks)
+    for hi, h in enumerate(hs):
+        _check_stats(p, ref, 0, hi, h, 1e-4)
+        bad, ties = compare_selection(p.sel[0, h].cpu().numpy(), ref["sel"][0, hi], ref["r"][0, hi], w.keep_k)
+        assert not bad, f"{name} head {h}: selection rows differ beyond ties: {bad[:10]}"
+        o2 = _attention_with(p, qkv, ref["sel"][0, hi], 0, h, o)
+        assert_output(_np(o2[0, h])[rows], ref["o"][0, hi][rows], "bf16", what=f"{name} head {h} oracle selection")
+
+
 EDGE = [
     # dtype, grid, text, block, keep_k, lam, mode
     ("bf16", (10, 10, 10), 0, 64, 0, 0.5, C.PISA_MODE_PISA),

@@ -103,6 +103,12 @@ __device__ __forceinline__ void fill_indicator(SmemA& sm, int block) {
   }
 }
 
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // max over the 8 bf16 of a 16-byte chunk of |x|, as the bit pattern of a non-negative bf16 in each
 // half of the result (clearing the sign makes the bit order the value order)
 __device__ __forceinline__ uint32_t absmax8(const uint4& u, uint32_t m) {
@@ -254,26 +260,34 @@ __device__ __forceinline__ void stats_a_body(const KVMaps& maps, const PreParams
         ok = !epi_any_failed(!wait_bar(&sm.full[s], (g >> 1) & 1, &sm.abort, p.status, p.wait_ns));
         if (!ok) break;
         // max |v| over the tile (and, zeroth order only, the fp16 value operand with scale 1):
-        // 16-byte chunks of the swizzled V tile, consecutive chunks per thread.  Rows past the group
-        // (or L) are zero or belong to no block of this group; they cannot raise the max above a
-        // real |v| of the head, but they are skipped all the same.
-        {
+        // 16-byte chunks of the swizzled V tile, consecutive chunks per thread.  A tile reaches past
+        // its group only at the end of the head, where the tile load fills zeros, so the maximum
+        // needs no row bound (only the head's maximum is used): the first-order sweep is unrolled
+        // into four independent running maxima.
+        if constexpr (kFirstOrder) {
+          uint32_t m4[4] = {vabs, 0u, 0u, 0u};
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int qq = tid + 128 * x, row = qq >> 4, c = qq & 15;
+            const uint4 uu = *reinterpret_cast<const uint4*>(sm.v[s] + (c >> 3) * kHalf + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+            m4[x & 3] = absmax8(uu, m4[x & 3]);
+          }
+          vabs = max_u16x2(max_u16x2(m4[0], m4[1]), max_u16x2(m4[2], m4[3]));
+        } else {
           const int rbase = gr.row0 + t * 128;
           for (int qq = tid; qq < 128 * 16; qq += 128) {
             const int row = qq >> 4, c = qq & 15;
             if (rbase + row >= gr.row1) break;
             const uint4 uu = *reinterpret_cast<const uint4*>(sm.v[s] + (c >> 3) * kHalf + row * 128 + (((c & 7) ^ (row & 7)) << 4));
             vabs = absmax8(uu, vabs);
-            if constexpr (!kFirstOrder) {
-              const uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
-              uint32_t hw[4];
+            const uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
+            uint32_t hw[4];
 #pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                const __half2 h2 = __floats2half2_rn(__uint_as_float(w[x] << 16), __uint_as_float(w[x] & 0xffff0000u));
-                hw[x] = *reinterpret_cast<const uint32_t*>(&h2);
-              }
-              *reinterpret_cast<uint4*>(vop + (size_t)(rbase + row) * D + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            for (int x = 0; x < 4; ++x) {
+              const __half2 h2 = __floats2half2_rn(__uint_as_float(w[x] << 16), __uint_as_float(w[x] & 0xffff0000u));
+              hw[x] = *reinterpret_cast<const uint32_t*>(&h2);
             }
+            *reinterpret_cast<uint4*>(vop + (size_t)(rbase + row) * D + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           }
         }
         mbar_arrive(&sm.empty[s]);
@@ -515,12 +529,12 @@ __device__ __forceinline__ void cov_norm_body(const KVMaps& maps, const PreParam
         {
           // fp16 copy of this tile's values, v / vscale: the H_j MMAs of the tile are done, so the
           // stage has landed and is held until the arrival below; 16-byte chunks, consecutive per
-          // thread
+          // thread, unrolled (the row bound only bites in the last tile of a head)
           const uint8_t* vt = sm.v[g % kStagesB];
           const int rbase = gr.row0 + t * 128;
-          for (int q = a; q < 128 * 16; q += 128) {
-            const int row = q >> 4, c = q & 15;
-            if (rbase + row >= gr.row1) break;
+#pragma unroll 4
+          for (int it = 0; it < 16; ++it) {
+            const int q = a + 128 * it, row = q >> 4, c = q & 15;
             const uint4 uu = *reinterpret_cast<const uint4*>(vt + (c >> 3) * kHalf + row * 128 + (((c & 7) ^ (row & 7)) << 4));
             const uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
             uint32_t hw[4];
@@ -533,7 +547,8 @@ __device__ __forceinline__ void cov_norm_body(const KVMaps& maps, const PreParam
               }
               hw[x] = pack_f16x2(lo, hi);
             }
-            *reinterpret_cast<uint4*>(vop + (size_t)(rbase + row) * D + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            if (rbase + row < gr.row1)
+              *reinterpret_cast<uint4*>(vop + (size_t)(rbase + row) * D + c * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           }
           mbar_arrive(&sm.empty[g % kStagesB]);
         }

@@ -21,7 +21,8 @@ PISA_DEVERR_WAIT_TIMEOUT, PISA_DEVERR_BAD_SELECTION = 1, 2
 SYMBOLS = ("pisa_abi_version", "pisa_num_blocks", "pisa_stats_bytes", "pisa_stats_carve", "pisa_workspace_bytes",
            "pisa_precompute", "pisa_route", "pisa_attention", "pisa_read_device_error", "pisa_status_string",
            "pisa_precompute_noalloc", "pisa_testing_set_attention_fault", "pisa_perblock_workspace_bytes",
-           "pisa_permute_rows", "pisa_axis_permutation", "pisa_precompute_zeroth_order", "pisa_precompute_route")
+           "pisa_permute_rows", "pisa_axis_permutation", "pisa_precompute_zeroth_order", "pisa_precompute_route",
+           "pisa_testing_set_precompute_fault")
 
 
 class PisaShape(ctypes.Structure):
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "pisa_status_string": (ctypes.c_char_p, [i32]),
             "pisa_precompute_noalloc": (i32, [P(PisaShape), vp, vp, vp, P(PisaStats), vp]),
             "pisa_testing_set_attention_fault": (i32, [i32, ctypes.c_uint64]),
+            "pisa_testing_set_precompute_fault": (i32, [i32, ctypes.c_uint64]),
             "pisa_permute_rows": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp]),
             "pisa_axis_permutation": (i32, [i32, i32, i32, i32, ctypes.c_char_p, P(i32), ctypes.c_int64]),
         }

@@ -13,6 +13,8 @@ constexpr int kMaxBlocks = 4096;
 // test-only fault injection (pisa_testing.h)
 int g_test_fault = PISA_TESTING_FAULT_NONE;
 unsigned long long g_test_wait_ns = 0;
+int g_test_pre_fault = PISA_TESTING_FAULT_NONE;
+unsigned long long g_test_pre_wait_ns = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -107,7 +109,7 @@ using namespace pisa;
 
 extern "C" {
 
-int32_t pisa_abi_version(void) { return 6; }
+int32_t pisa_abi_version(void) { return 7; }
 
 int32_t pisa_num_blocks(int32_t seq_len, int32_t block) {
   if (seq_len < 1 || block < 1) return -1;
@@ -186,7 +188,8 @@ pisa_status precompute(const pisa_shape* shape, const void* q, const void* k, co
   if (!ws || !aligned16(ws) || ws_bytes < pisa_workspace_bytes(shape)) return PISA_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (bf16_inputs(g.dtype)) {
-    cudaError_t e = launch_precompute_sm100(g, q, k, v, *stats, ws, first_order, cs);
+    cudaError_t e = launch_precompute_sm100(g, q, k, v, *stats, ws, first_order,
+                                            g_test_pre_wait_ns ? g_test_pre_wait_ns : kWaitLimitNs, g_test_pre_fault, cs);
     if (e == cudaSuccess && g.dtype == PISA_BF16_FP8QK) e = launch_quantize_fp8(g, q, k, *stats, cs);
     return cuda_status(e);
   }
@@ -362,6 +365,13 @@ pisa_status pisa_testing_set_attention_fault(int32_t fault, uint64_t wait_limit_
   if (fault != PISA_TESTING_FAULT_NONE && fault != PISA_TESTING_FAULT_SKIP_Q_LOAD) return PISA_ERR_INVALID_ARG;
   g_test_fault = fault;
   g_test_wait_ns = wait_limit_ns;
+  return PISA_OK;
+}
+
+pisa_status pisa_testing_set_precompute_fault(int32_t fault, uint64_t wait_limit_ns) {
+  if (fault != PISA_TESTING_FAULT_NONE && fault != PISA_TESTING_FAULT_SKIP_TILE_LOAD) return PISA_ERR_INVALID_ARG;
+  g_test_pre_fault = fault;
+  g_test_pre_wait_ns = wait_limit_ns;
   return PISA_OK;
 }
 

@@ -104,8 +104,11 @@ pisa_status validate_precompute(const pisa_shape* shape, const void* q, const vo
 // first_order = false: the zeroth-order statistics only (pisa_precompute_zeroth_order).
 cudaError_t launch_precompute_simt(const Dims& g, const void* q, const void* k, const void* v,
                                    const pisa_stats& st, void* ws, bool first_order, cudaStream_t stream);
+// wait_ns: the kernels' bounded-wait limit; fault: test-only fault injection (pisa_testing.h), 0
+// in normal calls.
 cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v,
-                                    const pisa_stats& st, void* ws, bool first_order, cudaStream_t stream);
+                                    const pisa_stats& st, void* ws, bool first_order,
+                                    unsigned long long wait_ns, int fault, cudaStream_t stream);
 // pdl: launch with programmatic stream serialization (the kernel waits for the previous kernel of
 // the stream before it reads anything, and lets the next one start at once).
 cudaError_t launch_hbar_reduce(const Dims& g, const float* partials, int nparts, const float* vmax,

@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(256) value_scale_finish(const __nv_bfloat16* _
 }  // namespace
 
 cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k, const void* v, const pisa_stats& st,
-                                    void* ws, bool first_order, cudaStream_t stream) {
+                                    void* ws, bool first_order, unsigned long long wait_ns, int fault,
+                                    cudaStream_t stream) {
   KVMaps maps;
   const uint64_t bh = (uint64_t)g.BH();
   if (!encode_bf16_3d(&maps.q, q, D, g.L, bh, 128) || !encode_bf16_3d(&maps.k, k, D, g.L, bh, 128) ||
@@ -136,7 +137,8 @@ cudaError_t launch_precompute_sm100(const Dims& g, const void* q, const void* k,
   p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kStatusBytes);
   p.vmax = reinterpret_cast<float*>(static_cast<char*>(ws) + vmax_offset(g));
   p.status = static_cast<int*>(ws);
-  p.wait_ns = kWaitLimitNs;
+  p.wait_ns = wait_ns;
+  p.fault = fault;
   const size_t smem_a = sizeof(SmemA) + 1024, smem_b = sizeof(SmemB) + 1024;
   cudaError_t e;
   if ((e = set_max_dynamic_smem(reinterpret_cast<const void*>(stats_a_sm100<true>), smem_a))) return e;

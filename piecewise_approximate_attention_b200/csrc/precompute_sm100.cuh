@@ -55,6 +55,7 @@ struct PreParams {
   float* vmax;               // [BH][nparts] max |v| per group (pass A)
   int* status;
   unsigned long long wait_ns;
+  int fault = 0;             // test-only fault injection (pisa_testing.h); 0 in normal calls
 };
 
 // ----------------------------------------------------------------------------------------------
@@ -181,11 +182,14 @@ __device__ __forceinline__ void stats_a_body(const KVMaps& maps, const PreParams
     if (lane == 0) {
       int g = 0;
       bool ok = true;
+      // fault 2 (tests only): the first tile is never loaded, so the MMA warp's wait for it runs out
+      const int skipped = p.fault == 2 ? 0 : -1;
       for (int u = u0; u < u1 && ok; ++u) {
         const Group gr = group_of(p, u, ngroups);
         for (int t = 0; t < gr.ntile; ++t, ++g) {
           const int s = g & 1;
           if (g >= 2 && !(ok = wait_bar(&sm.empty[s], ((g >> 1) - 1) & 1, &sm.abort, p.status, p.wait_ns))) break;
+          if (g == skipped) continue;
           const int y = gr.row0 + t * 128;
           mbar_expect_tx(&sm.full[s], 3 * kTile);
           tma_load_3d(sm.q[s], &maps.q, &sm.full[s], 0, y, gr.bh);
@@ -197,7 +201,8 @@ __device__ __forceinline__ void stats_a_body(const KVMaps& maps, const PreParams
         }
       }
       {   // let issued copies land before shared memory is released (normally already landed)
-        for (int i = max(0, g - 2); i < g; ++i) mbar_drain(&sm.full[i & 1], (i >> 1) & 1, p.wait_ns);
+        for (int i = max(0, g - 2); i < g; ++i)
+          if (i != skipped) mbar_drain(&sm.full[i & 1], (i >> 1) & 1, p.wait_ns);
       }
     }
   } else if (warp == 5) {

@@ -30,7 +30,7 @@ int main(void) {
   int32_t perm[25];
   int32_t i, seen[25] = {0};
 
-  CHECK(1, pisa_abi_version() == 6);
+  CHECK(1, pisa_abi_version() == 7);
   CHECK(2, pisa_num_blocks(75600, 128) == 591);
   CHECK(3, pisa_num_blocks(0, 64) == -1);
 

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_blocks():
-    assert C.lib().pisa_abi_version() == 6
+    assert C.lib().pisa_abi_version() == 7
     assert C.pisa_num_blocks(32760, 64) == 512
     assert C.pisa_num_blocks(75600, 128) == 591
     assert C.pisa_num_blocks(1, 64) == 1
@@ -194,6 +194,10 @@ def test_missing_library_fails_loudly(monkeypatch):
 def test_testing_hook_rejects_unknown_fault():
     assert C.lib().pisa_testing_set_attention_fault(7, 0) == C.PISA_ERR_INVALID_ARG
     assert C.lib().pisa_testing_set_attention_fault(0, 0) == C.PISA_OK
+    # the pre-computation hook takes its own fault code only
+    assert C.lib().pisa_testing_set_precompute_fault(1, 0) == C.PISA_ERR_INVALID_ARG
+    assert C.lib().pisa_testing_set_precompute_fault(7, 0) == C.PISA_ERR_INVALID_ARG
+    assert C.lib().pisa_testing_set_precompute_fault(0, 0) == C.PISA_OK
 
 
 def test_reordering_entry_points_validate_without_launch():
@@ -234,7 +238,7 @@ def test_headers_are_plain_c_and_the_library_links_from_c(tmp_path):
                     f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
     res = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0, res.stderr
-    assert "c consumer ok: abi 6" in res.stdout
+    assert "c consumer ok: abi 7" in res.stdout
 
 
 def test_precompute_route_checks_its_flags():

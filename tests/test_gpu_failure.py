@@ -50,6 +50,48 @@ def test_wait_timeout_is_reported_and_context_survives():
     assert_output(o2[0, 0].double().cpu().numpy()[keep], ref["o"][0, 0][keep], "bf16", what="after timeout")
 
 
+SKIP_TILE_LOAD = 2
+
+
+@pytest.mark.parametrize("first_order", [True, False], ids=["first_order", "zeroth_order"])
+def test_precompute_wait_timeout_is_reported_and_context_survives(first_order):
+    """The pre-computation's first pass never gets the first tile of each CTA's first group: with
+    10 heads x 16 groups (more groups than SMs, so several CTAs own two) every CTA's bounded wait
+    runs out and it must give up all its groups, drain and return; the reduction and the second
+    pass, launched as its programmatic dependents, must still end.  The status word reports the
+    timeout, and the next call on the context runs normally and matches the oracle."""
+    w = Workload("fault", 1, 10, (4, 64, 128), 0, 128, 128, 0.875, 0.5, "bf16", seed=4)
+    q, k, v = make_qkv(w)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    lam = w.lam if first_order else 0.0
+    mode = C.PISA_MODE_PISA if first_order else C.PISA_MODE_EXACT_ONLY
+    p = Pisa(1, w.heads, w.seq_len, 128, w.block, w.keep_k, lam, "bf16", 1.0, "cuda", mode, first_order=first_order)
+    assert C.lib().pisa_testing_set_precompute_fault(SKIP_TILE_LOAD, WAIT_NS) == C.PISA_OK
+    try:
+        p.precompute(qd, kd, vd)
+        torch.cuda.synchronize()
+    finally:
+        assert C.lib().pisa_testing_set_precompute_fault(0, 0) == C.PISA_OK
+    assert p.device_error() == (C.PISA_ERR_DEVICE_TIMEOUT, C.PISA_DEVERR_WAIT_TIMEOUT)
+    assert p.device_error() == (C.PISA_OK, 0)
+    p.precompute(qd, kd, vd)
+    p.route()
+    o = torch.empty_like(qd)
+    p.attention(qd, kd, vd, o)
+    torch.cuda.synchronize()
+    assert p.device_error() == (C.PISA_OK, 0)
+    hs = [0, 9]
+    md = "pisa" if first_order else "exact_only"
+    ref = O.pisa(q[:, hs].double().numpy(), k[:, hs].double().numpy(), v[:, hs].double().numpy(), w.block, w.keep_k,
+                 lam, mode=md, qblocks=[0, 100, 255])
+    rows = rows_of_blocks(w.seq_len, w.block, [0, 100, 255])
+    for hi, h in enumerate(hs):
+        bad, ties = compare_selection(p.sel[0, h].cpu().numpy(), ref["sel"][0, hi], ref["r"][0, hi], w.keep_k)
+        assert not bad
+        keep = rows & ~rows_of_blocks(w.seq_len, w.block, ties)
+        assert_output(o[0, h].double().cpu().numpy()[keep], ref["o"][0, hi][keep], "bf16", what=f"head {h} after timeout")
+
+
 @pytest.mark.parametrize("dtype,mode", [("bf16_fp8qk", C.PISA_MODE_PISA), ("bf16", C.PISA_MODE_PER_BLOCK)])
 def test_wait_timeout_in_other_paths(dtype, mode):
     """The same bounded wait in the e4m3-logit instantiation, and in the per-block mode, where the

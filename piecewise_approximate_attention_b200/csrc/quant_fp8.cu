@@ -4,7 +4,9 @@
 // nearest even and saturated, both computed in float32 (IEEE division).
 //
 // HBM-bound: q and k are read once more (bf16) and written as one byte per element.  One warp per
-// row, four elements per lane (a 128-element row is 256 bytes of bf16 in, 128 bytes of codes out).
+// row, four elements per lane (a 128-element row is 256 bytes of bf16 in, 128 bytes of codes out);
+// a warp issues the loads of several rows before it reduces any of them, so that enough bytes are
+// in flight to cover the memory latency.
 #include "common.cuh"
 
 namespace pisa {
@@ -52,13 +54,18 @@ __device__ __forceinline__ void store_codes(uint8_t* row, int lane, const float*
 __global__ void __launch_bounds__(kThreads) quant_rows(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ dst,
                                                       float* __restrict__ scale, int L) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, bh = blockIdx.y;
-  for (int r = (blockIdx.x * kWarps + warp) * kRowsPerWarp, e = 0; e < kRowsPerWarp && r < L; ++e, ++r) {
-    const size_t row = (size_t)bh * L + r;
-    float x[4];
-    load4(src + row * 128, lane, x);
-    const float amax = warp_absmax(x);
+  const int r0 = (blockIdx.x * kWarps + warp) * kRowsPerWarp;
+  float x[kRowsPerWarp][4];
+#pragma unroll
+  for (int e = 0; e < kRowsPerWarp; ++e)
+    if (r0 + e < L) load4(src + ((size_t)bh * L + r0 + e) * 128, lane, x[e]);
+#pragma unroll
+  for (int e = 0; e < kRowsPerWarp; ++e) {
+    if (r0 + e >= L) break;
+    const size_t row = (size_t)bh * L + r0 + e;
+    const float amax = warp_absmax(x[e]);
     const float s = amax > 0.f ? amax / kE4m3Max : 1.f;
-    store_codes(dst + row * 128, lane, x, s);
+    store_codes(dst + row * 128, lane, x[e], s);
     if (lane == 0) scale[row] = s;
   }
 }
@@ -72,20 +79,29 @@ __global__ void __launch_bounds__(kThreads) quant_groups(const T* __restrict__ s
   const int r0 = blockIdx.x * group, r1 = min(rows, r0 + group);
   const size_t base = (size_t)bh * rows;
   float m = 0.f;
-  for (int r = r0 + warp; r < r1; r += kWarps) {
-    float x[4];
-    load4(src + (base + r) * 128, lane, x);
-    m = fmaxf(m, warp_absmax(x));
+  // the maximum over the group's rows, four rows of a warp in flight at once
+  for (int r = r0 + warp; r < r1; r += 4 * kWarps) {
+    float x[4][4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (r + e * kWarps < r1) load4(src + (base + r + e * kWarps) * 128, lane, x[e]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (r + e * kWarps < r1) m = fmaxf(m, warp_absmax(x[e]));
   }
   if (lane == 0) red[warp] = m;
   __syncthreads();
   float amax = 0.f;
   for (int w = 0; w < kWarps; ++w) amax = fmaxf(amax, red[w]);
   const float s = amax > 0.f ? amax / kE4m3Max : 1.f;
-  for (int r = r0 + warp; r < r1; r += kWarps) {
-    float x[4];
-    load4(src + (base + r) * 128, lane, x);
-    store_codes(dst + (base + r) * 128, lane, x, s);
+  for (int r = r0 + warp; r < r1; r += 4 * kWarps) {
+    float x[4][4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (r + e * kWarps < r1) load4(src + (base + r + e * kWarps) * 128, lane, x[e]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (r + e * kWarps < r1) store_codes(dst + (base + r + e * kWarps) * 128, lane, x[e], s);
   }
   if (threadIdx.x == 0) scale[(size_t)bh * gridDim.x + blockIdx.x] = s;
 }
